@@ -1,0 +1,149 @@
+// Head-specific MLP estimator and tile scores (Veda summary 2.1,
+// Head-Specific Projections).
+//
+//   emb = W2^T GELU(W1^T desc + b1) + b2   per tile, per head, for Q and K
+//   scores[i, j] = scale * emb_q[i] . emb_k[j]
+//
+// Two kernels, both fp32 FFMA (no TF32): an MLP kernel that keeps 32 tile
+// descriptors in shared memory and streams each weight once per CTA, and a
+// 64x64-tiled SGEMM for the score matrix. The embeddings live in the
+// caller's scratch buffer between the two.
+#include "veda_internal.cuh"
+
+namespace veda {
+namespace {
+
+constexpr int MLP_ROWS = 32;
+
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+
+// grid (ceil(nt_cap/32), heads, B*2): z%2 == 0 -> query side, 1 -> key side.
+__global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerGeom g, const float* __restrict__ dq,
+                                                  const float* __restrict__ dk, const float* __restrict__ w1q,
+                                                  const float* __restrict__ b1q, const float* __restrict__ w2q,
+                                                  const float* __restrict__ b2q, const float* __restrict__ w1k,
+                                                  const float* __restrict__ b1k, const float* __restrict__ w2k,
+                                                  const float* __restrict__ b2k, int hidden, int out_dim,
+                                                  float* __restrict__ emb) {
+  extern __shared__ float sm[];
+  const int din = 3 * g.d;
+  float* xs = sm;                          // [MLP_ROWS][din]
+  float* hs = sm + MLP_ROWS * din;         // [MLP_ROWS][hidden]
+  const int h = blockIdx.y;
+  const int b = blockIdx.z >> 1;
+  const int side = blockIdx.z & 1;
+  const int r0 = blockIdx.x * MLP_ROWS;
+  const int nt = g.h[h].nt;
+  const float* desc = (side ? dk : dq) + (((long long)b * g.heads + h) * g.nt_cap) * din;
+  const float* W1 = (side ? w1k : w1q) + (long long)h * din * hidden;
+  const float* B1 = (side ? b1k : b1q) + (long long)h * hidden;
+  const float* W2 = (side ? w2k : w2q) + (long long)h * hidden * out_dim;
+  const float* B2 = (side ? b2k : b2q) + (long long)h * out_dim;
+  float* out = emb + ((long long)side * g.B * g.heads + (long long)b * g.heads + h) * g.nt_cap * out_dim;
+
+  for (int i = threadIdx.x; i < MLP_ROWS * din; i += blockDim.x) {
+    const int r = i / din, c = i - r * din;
+    xs[i] = (r0 + r < nt) ? desc[(long long)(r0 + r) * din + c] : 0.f;
+  }
+  __syncthreads();
+  // layer 1 + GELU: thread owns hidden units j, j+128
+  for (int j = threadIdx.x; j < hidden; j += blockDim.x) {
+    float acc[MLP_ROWS];
+    const float bj = B1[j];
+#pragma unroll
+    for (int r = 0; r < MLP_ROWS; ++r) acc[r] = bj;
+    for (int i = 0; i < din; ++i) {
+      const float w = __ldg(W1 + (long long)i * hidden + j);
+#pragma unroll
+      for (int r = 0; r < MLP_ROWS; ++r) acc[r] = fmaf(xs[r * din + i], w, acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < MLP_ROWS; ++r) hs[r * hidden + j] = gelu_erf(acc[r]);
+  }
+  __syncthreads();
+  // layer 2
+  for (int j = threadIdx.x; j < out_dim; j += blockDim.x) {
+    float acc[MLP_ROWS];
+    const float bj = B2[j];
+#pragma unroll
+    for (int r = 0; r < MLP_ROWS; ++r) acc[r] = bj;
+    for (int i = 0; i < hidden; ++i) {
+      const float w = __ldg(W2 + (long long)i * out_dim + j);
+#pragma unroll
+      for (int r = 0; r < MLP_ROWS; ++r) acc[r] = fmaf(hs[r * hidden + i], w, acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < MLP_ROWS; ++r)
+      if (r0 + r < g.nt_cap) out[(long long)(r0 + r) * out_dim + j] = (r0 + r < nt) ? acc[r] : 0.f;
+  }
+}
+
+// scores[b,h,i,j] = scale * q[i].k[j]; 64x64 output tile per CTA, 4x4 per thread.
+__global__ void __launch_bounds__(256) score_gemm_kernel(const __grid_constant__ LayerGeom g, const float* __restrict__ emb,
+                                                         int out_dim, float scale, float* __restrict__ scores) {
+  __shared__ float As[32][64 + 4];
+  __shared__ float Bs[32][64 + 4];
+  const int h = blockIdx.z % g.heads;
+  const int b = blockIdx.z / g.heads;
+  const int nt = g.h[h].nt;
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  const long long bh = (long long)b * g.heads + h;
+  const float* Q = emb + bh * g.nt_cap * out_dim;
+  const float* K = emb + ((long long)g.B * g.heads + bh) * g.nt_cap * out_dim;
+  float* C = scores + bh * (long long)g.nt_cap * g.nt_cap;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  if (i0 < nt && j0 < nt) {
+    for (int e0 = 0; e0 < out_dim; e0 += 32) {
+      for (int t = threadIdx.x; t < 64 * 32; t += 256) {
+        const int r = t / 32, e = t % 32;
+        const bool ein = e0 + e < out_dim;
+        As[e][r] = (i0 + r < nt && ein) ? Q[(long long)(i0 + r) * out_dim + e0 + e] : 0.f;
+        Bs[e][r] = (j0 + r < nt && ein) ? K[(long long)(j0 + r) * out_dim + e0 + e] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int e = 0; e < 32; ++e) {
+        const float4 a = *reinterpret_cast<const float4*>(&As[e][ty * 4]);
+        const float4 bb = *reinterpret_cast<const float4*>(&Bs[e][tx * 4]);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+      }
+      __syncthreads();
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = i0 + ty * 4 + u;
+    if (i >= g.nt_cap) continue;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = j0 + tx * 4 + w;
+      if (j < g.nt_cap) C[(long long)i * g.nt_cap + j] = (i < nt && j < nt) ? acc[u][w] * scale : 0.f;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_tile_scores(const LayerGeom& g, const float* dq, const float* dk, const float* w1q,
+                               const float* b1q, const float* w2q, const float* b2q, const float* w1k,
+                               const float* b1k, const float* w2k, const float* b2k, int hidden, int out_dim,
+                               float scale, float* scores, float* emb_ws, cudaStream_t s) {
+  const size_t smem = (size_t)MLP_ROWS * (3 * g.d + hidden) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 g1((g.nt_cap + MLP_ROWS - 1) / MLP_ROWS, g.heads, g.B * 2);
+  mlp_kernel<<<g1, 128, smem, s>>>(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int nb = (g.nt_cap + 63) / 64;
+  const dim3 g2(nb, nb, g.heads * g.B);
+  score_gemm_kernel<<<g2, 256, 0, s>>>(g, emb_ws, out_dim, scale, scores);
+  return cudaGetLastError();
+}
+
+}  // namespace veda

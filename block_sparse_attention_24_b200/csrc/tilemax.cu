@@ -1,0 +1,349 @@
+// Oracle tile map and row-wise KL (Veda summary 2.1, Target Construction and
+// Optimization; 2.3, Training Efficiency: the heat map is built in two
+// passes, on a subset of query tiles).
+//
+// One CTA owns 128 query rows (one 128-token query tile, or two 64-token
+// query tiles) of one selected head and sweeps every key block of the head
+// twice with tcgen05 S = Q K^T:
+//   pass 1: per row, lse = log2-domain log-sum-exp over all valid keys;
+//   pass 2: per row and key tile, the largest logit minus lse, then the
+//           maximum over the tile's valid rows (warp shuffle, then a shared
+//           order-preserving atomicMax) -> M[a, b] = exp2(.) = max-pooled
+//           softmax probability over the tile region.
+// Roles as in the attention kernel: 4 softmax warps (row r = TMEM lane r), a
+// TMA producer warp with a 3-stage K ring, one MMA-issuing thread, S double
+// buffered in TMEM. A second kernel turns map rows and score rows into KL
+// values, a third averages them in a fixed order.
+#include "veda_internal.cuh"
+
+namespace veda {
+namespace {
+
+constexpr int BM = 128, BN = 128;
+constexpr int KST = 3;  // K ring stages
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int NUM_THREADS = 192;
+
+template <int D>
+struct MapLayout {
+  static constexpr int QB = BM * D * 2;
+  static constexpr int KB = BN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = QB;
+  static constexpr int OFF_BAR = OFF_K + KST * KB;
+  static constexpr int NUM_BARS = 1 + 2 * KST + 2 + 2 + 1;  // q_full, k_full/empty, s_full, s_free, drain
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_PART = (OFF_MISC + 16 + 15) / 16 * 16;
+  static int bytes(int nt_cap) { return OFF_PART + (BM / 64) * nt_cap * 4 + 1024; }
+};
+
+struct MapParams {
+  float scale_log2;
+  int n_rows;
+  const int32_t* rows;  // [n_heads_sel, n_rows] or NULL
+  float* tilemap;       // [n_heads_sel, n_rows, nt_cap]
+  float* lse;           // [n_heads_sel, n_rows, tile] or NULL
+  int heads_sel[VEDA_MAX_HEADS];
+};
+
+__device__ __forceinline__ uint32_t ord_f32(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unord_f32(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+template <int D, int TILE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tilemax_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ MapParams prm) {
+  using Lay = MapLayout<D>;
+  constexpr int NSUB = BM / TILE;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+
+  const int hs = blockIdx.y;
+  const int h = prm.heads_sel[hs];
+  const int bh = h;  // B == 1
+  const HeadGeom& hg = g.h[h];
+  const int nt = hg.nt;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_kb = (nt * TILE + BN - 1) / BN;
+  const int iters = 2 * n_kb;
+
+  // query tiles of this CTA
+  int qt[NSUB];
+  bool qv[NSUB];
+#pragma unroll
+  for (int s = 0; s < NSUB; ++s) {
+    const int r = blockIdx.x * NSUB + s;
+    qv[s] = r < prm.n_rows;
+    int a = qv[s] ? (prm.rows ? __ldg(prm.rows + (long long)hs * prm.n_rows + r) : r) : 0;
+    if (a < 0 || a >= nt) {
+      if (qv[s]) report(g.dev_status, VEDA_ERR_BAD_INDEX);
+      a = 0;
+      qv[s] = false;
+    }
+    qt[s] = a;
+  }
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 1 + KST;
+  uint64_t* s_full = bars + 1 + 2 * KST;
+  uint64_t* s_free = bars + 3 + 2 * KST;
+  uint64_t* drain = bars + 5 + 2 * KST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
+  uint32_t* part = reinterpret_cast<uint32_t*>(smem + Lay::OFF_PART);  // [NSUB][nt_cap] ordered maxima
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < Lay::NUM_BARS; ++i) mbar_init(bars + i, (i == 3 + 2 * KST || i == 4 + 2 * KST) ? 128 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < NSUB * g.nt_cap; i += NUM_THREADS) part[i] = 0u;  // 0 = no contribution
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      mbar_expect_tx(q_full, Lay::QB);
+#pragma unroll
+      for (int s = 0; s < NSUB; ++s)
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(smem + Lay::OFF_Q + bx * BM * 128 + s * TILE * 128, &tmQ, q_full, bx * 64, qt[s] * TILE, bh);
+      int issued = 0;
+      for (int it = 0; it < iters; ++it) {
+        const int st = it % KST;
+        if (it >= KST && !mbar_wait(k_empty + st, ((it - KST) / KST) & 1, abort_flag, g.dev_status)) break;
+        mbar_expect_tx(k_full + st, Lay::KB);
+        const int kb = it % n_kb;
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(smem + Lay::OFF_K + st * Lay::KB + bx * BN * 128, &tmK, k_full + st, bx * 64, kb * BN, bh);
+        issued = it + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait_drain(q_full, 0, VEDA_WAIT_LIMIT_NS);
+        for (int it = issued - KST < 0 ? 0 : issued - KST; it < issued; ++it)
+          mbar_wait_drain(k_full + it % KST, (it / KST) & 1, VEDA_WAIT_LIMIT_NS);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
+      const uint32_t aQ = smem_u32(smem + Lay::OFF_Q);
+      const uint32_t aK = smem_u32(smem + Lay::OFF_K);
+      if (mbar_wait(q_full, 0, abort_flag, g.dev_status)) {
+        tc_fence_after();
+        for (int it = 0; it < iters; ++it) {
+          const int s = it & 1, st = it % KST;
+          if (it >= 2 && !mbar_wait(s_free + s, ((it - 2) >> 1) & 1, abort_flag, g.dev_status)) break;
+          if (!mbar_wait(k_full + st, (it / KST) & 1, abort_flag, g.dev_status)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+            umma_bf16_ss(tmem + s * BN, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + st * Lay::KB + off, 16, 1024),
+                         idesc, kk > 0);
+          }
+          umma_commit(s_full + s);
+          umma_commit(k_empty + st);
+        }
+      }
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, VEDA_WAIT_LIMIT_NS);
+    }
+  } else {
+    const int r = threadIdx.x;
+    const int qs = r / TILE;  // query sub-tile of this row
+    const bool row_valid = qv[qs] && (r % TILE) < tile_len(hg, g.T, qt[qs]);
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const float C = prm.scale_log2;
+    float m = -INFINITY, l = 0.f, lse2 = 0.f;
+    for (int it = 0; it < iters; ++it) {
+      const int s = it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (it >> 1) & 1, abort_flag, g.dev_status))) break;
+      tc_fence_after();
+      float sv[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(lane_addr + s * BN + c * 32, u);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free + s);  // S buffer may be overwritten now
+      const int kb = it % n_kb;
+      const bool pass2 = it >= n_kb;
+#pragma unroll
+      for (int u = 0; u < NSUB; ++u) {
+        const int kt = kb * NSUB + u;
+        const int klen = kt < nt ? tile_len(hg, g.T, kt) : 0;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < TILE; ++c) mx = fmaxf(mx, c < klen ? sv[u * TILE + c] : -INFINITY);
+        if (!pass2) {
+          if (klen > 0) {
+            const float mnew = fmaxf(m, mx * C);
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < TILE; ++c) acc += c < klen ? fast_exp2(fmaf(sv[u * TILE + c], C, -mnew)) : 0.f;
+            l = l * fast_exp2(m - mnew) + acc;
+            m = mnew;
+          }
+        } else {
+          float v = (row_valid && klen > 0) ? fmaf(mx, C, -lse2) : -INFINITY;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+          if (lane == 0 && kt < nt && v > -INFINITY) atomicMax(part + qs * g.nt_cap + kt, ord_f32(v));
+        }
+      }
+      if (it == n_kb - 1) {
+        lse2 = m + __log2f(l);
+        const int rr = blockIdx.x * NSUB + qs;
+        if (prm.lse && rr < prm.n_rows)
+          prm.lse[((long long)hs * prm.n_rows + rr) * TILE + (r % TILE)] = row_valid ? lse2 * 0.69314718055994531f : 0.f;
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+  // write the map rows and lse
+  if (!*abort_flag) {
+#pragma unroll
+    for (int s = 0; s < NSUB; ++s) {
+      const int rr = blockIdx.x * NSUB + s;
+      if (rr >= prm.n_rows) continue;
+      float* out = prm.tilemap + ((long long)hs * prm.n_rows + rr) * g.nt_cap;
+      for (int b = threadIdx.x; b < g.nt_cap; b += NUM_THREADS) {
+        const uint32_t k = part[s * g.nt_cap + b];
+        out[b] = (b < nt && k != 0u && qv[s]) ? fast_exp2(unord_f32(k)) : 0.f;
+      }
+    }
+  }
+}
+
+__global__ void kl_rows_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ MapParams prm,
+                               int n_heads_sel, const float* __restrict__ scores, float* __restrict__ kl_rows) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32, lane = threadIdx.x % 32;
+  if (warp >= n_heads_sel * prm.n_rows) return;
+  const int hs = warp / prm.n_rows, rr = warp % prm.n_rows;
+  const int h = prm.heads_sel[hs];
+  const int nt = g.h[h].nt;
+  int a = prm.rows ? __ldg(prm.rows + (long long)hs * prm.n_rows + rr) : rr;
+  if (a < 0 || a >= nt) {
+    if (lane == 0) kl_rows[warp] = 0.f;
+    return;
+  }
+  const float* M = prm.tilemap + (long long)warp * g.nt_cap;
+  const float* S = scores + ((long long)h * g.nt_cap + a) * g.nt_cap;
+  float msum = 0.f, smax = -INFINITY;
+  for (int b = lane; b < nt; b += 32) {
+    msum += M[b];
+    smax = fmaxf(smax, S[b]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    msum += __shfl_xor_sync(0xffffffffu, msum, off);
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
+  }
+  float z = 0.f;
+  for (int b = lane; b < nt; b += 32) z += expf(S[b] - smax);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+  const float logz = logf(z), log_msum = logf(msum);
+  float kl = 0.f;
+  for (int b = lane; b < nt; b += 32) {
+    const float mb = M[b];
+    if (mb > 0.f) {
+      const float t = mb / msum;
+      kl += t * ((logf(mb) - log_msum) - (S[b] - smax - logz));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) kl += __shfl_xor_sync(0xffffffffu, kl, off);
+  if (lane == 0) kl_rows[warp] = kl;
+}
+
+__global__ void kl_mean_kernel(const float* __restrict__ kl_rows, int n_heads_sel, int n_rows, float* __restrict__ out) {
+  __shared__ float red[32];
+  float total = 0.f;
+  for (int hs = 0; hs < n_heads_sel; ++hs) {
+    float acc = 0.f;
+    for (int r = threadIdx.x; r < n_rows; r += blockDim.x) acc += kl_rows[(long long)hs * n_rows + r];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s = 0.f;
+      for (int w = 0; w < (int)(blockDim.x / 32); ++w) s += red[w];
+      total += s / (float)n_rows;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = total / (float)n_heads_sel;
+}
+
+template <int D, int TILE>
+cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, const MapParams& prm, int n_heads_sel,
+                         cudaStream_t s) {
+  CUtensorMap tq, tk;
+  const uint64_t rows = (uint64_t)g.n_cap, planes = (uint64_t)g.B * g.heads;
+  if (encode_tensor_map_3d_bf16(&tq, qp, D, rows, planes, 64, TILE) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_bf16(&tk, kp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto kern = tilemax_kernel<D, TILE>;
+  const int smem = MapLayout<D>::bytes(g.nt_cap);
+  if (smem > 232448) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((prm.n_rows + BM / TILE - 1) / (BM / TILE), n_heads_sel, 1);
+  kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, const int32_t* heads_sel,
+                           int n_heads_sel, const int32_t* rows, int n_rows, float scale, float* tilemap, float* lse,
+                           const float* scores, float* kl_rows, float* kl_out, cudaStream_t s) {
+  MapParams prm;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.n_rows = n_rows;
+  prm.rows = rows;
+  prm.tilemap = tilemap;
+  prm.lse = lse;
+  for (int i = 0; i < VEDA_MAX_HEADS; ++i) prm.heads_sel[i] = i < n_heads_sel ? heads_sel[i] : 0;
+  cudaError_t e;
+  if (g.d == 128 && g.tile == 128) e = launch_map_t<128, 128>(g, qp, kp, prm, n_heads_sel, s);
+  else if (g.d == 128 && g.tile == 64) e = launch_map_t<128, 64>(g, qp, kp, prm, n_heads_sel, s);
+  else if (g.d == 64 && g.tile == 128) e = launch_map_t<64, 128>(g, qp, kp, prm, n_heads_sel, s);
+  else e = launch_map_t<64, 64>(g, qp, kp, prm, n_heads_sel, s);
+  if (e != cudaSuccess || !scores) return e;
+  const int warps = n_heads_sel * n_rows;
+  kl_rows_kernel<<<(warps * 32 + 255) / 256, 256, 0, s>>>(g, prm, n_heads_sel, scores, kl_rows);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  kl_mean_kernel<<<1, 1024, 0, s>>>(kl_rows, n_heads_sel, n_rows, kl_out);
+  return cudaGetLastError();
+}
+
+}  // namespace veda

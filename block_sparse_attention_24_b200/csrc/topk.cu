@@ -1,0 +1,142 @@
+// Top-k key tiles per query tile (Veda summary 2.1 and 4: only the highest
+// scoring key tiles are kept).
+//
+// One warp per score row. The row is staged in shared memory as
+// order-preserving 32-bit keys (larger float -> larger key, -0.0 folded into
+// +0.0). A 4-pass, 8-bit radix select finds the exact k-th largest key T and
+// how many keys equal to T must be kept; a final pass in column order keeps
+// every key > T and the lowest-index keys == T, so exact ties go to the lower
+// tile index and the output list comes out ascending without a sort.
+// Histogram updates are warp-aggregated (__match_any_sync) shared atomics.
+#include "veda_internal.cuh"
+
+namespace veda {
+namespace {
+
+constexpr int TOPK_WARPS = 4;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (f == 0.0f) u = 0u;  // -0.0 ties +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_constant__ LayerGeom g,
+                                                               const float* __restrict__ scores, int k_cap,
+                                                               int32_t* __restrict__ idx, uint8_t* __restrict__ mask) {
+  extern __shared__ uint32_t sm_u32[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint32_t* keys = sm_u32 + warp * (g.nt_cap + 256);
+  uint32_t* hist = keys + g.nt_cap;
+  const long long rows = (long long)g.B * g.heads * g.nt_cap;
+  const long long row = (long long)blockIdx.x * TOPK_WARPS + warp;
+  if (row >= rows) return;
+  const int a = (int)(row % g.nt_cap);
+  const int h = (int)((row / g.nt_cap) % g.heads);
+  const int nt = g.h[h].nt;
+  const int k = g.h[h].k;
+  int32_t* idx_row = idx + row * k_cap;
+  uint8_t* mask_row = mask ? mask + row * g.nt_cap : nullptr;
+  if (a >= nt) {
+    for (int p = lane; p < k_cap; p += 32) idx_row[p] = -1;
+    if (mask_row)
+      for (int c = lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
+    return;
+  }
+  const float* srow = scores + row * g.nt_cap;
+  for (int c = lane; c < nt; c += 32) keys[c] = order_key(__ldg(srow + c));
+  __syncwarp();
+
+  uint32_t prefix = 0u, pmask = 0u;
+  int remaining = k;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0u;
+    __syncwarp();
+    for (int c0 = 0; c0 < nt; c0 += 32) {
+      const int c = c0 + lane;
+      const bool in = c < nt;
+      const uint32_t key = in ? keys[c] : 0u;
+      const bool match = in && ((key & pmask) == prefix);
+      const uint32_t active = __ballot_sync(0xffffffffu, match);
+      if (match) {
+        const uint32_t bin = (key >> shift) & 255u;
+        const uint32_t same = __match_any_sync(active, bin);
+        if ((__ffs(same) - 1) == lane) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+      }
+    }
+    __syncwarp();
+    // lane l owns bins 255-8l .. 248-8l (descending); scan from the top
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) cnt += hist[255 - 8 * lane - q];
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const uint32_t excl = incl - cnt;
+    const bool here = excl < (uint32_t)remaining && (uint32_t)remaining <= incl;
+    const uint32_t who = __ballot_sync(0xffffffffu, here);
+    const int L = __ffs(who) - 1;  // exactly one lane: the class holds >= remaining keys
+    uint32_t digit = 0, above = 0;
+    if (lane == L) {
+      uint32_t acc = excl;
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t bin = 255 - 8 * lane - q;
+        if (acc + hist[bin] >= (uint32_t)remaining) {
+          digit = bin;
+          above = acc;
+          break;
+        }
+        acc += hist[bin];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, L);
+    above = __shfl_sync(0xffffffffu, above, L);
+    remaining -= (int)above;
+    prefix |= digit << shift;
+    pmask |= 255u << shift;
+    __syncwarp();
+  }
+  // prefix is now the k-th largest key; keep all larger keys and the first
+  // `remaining` equal keys in column order.
+  const uint32_t T = prefix;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int base = 0, eq_seen = 0;
+  for (int c0 = 0; c0 < nt; c0 += 32) {
+    const int c = c0 + lane;
+    const bool in = c < nt;
+    const uint32_t key = in ? keys[c] : 0u;
+    const bool eq = in && key == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_seen + __popc(eqm & lt_mask);
+    const bool sel = in && (key > T || (eq && eq_rank < remaining));
+    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) idx_row[base + __popc(selm & lt_mask)] = c;
+    if (mask_row && in) mask_row[c] = sel ? 1 : 0;
+    base += __popc(selm);
+    eq_seen += __popc(eqm);
+  }
+  for (int p = k + lane; p < k_cap; p += 32) idx_row[p] = -1;
+  if (mask_row)
+    for (int c = nt + lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int32_t* idx, uint8_t* mask,
+                        cudaStream_t s) {
+  const size_t smem = (size_t)TOPK_WARPS * (g.nt_cap + 256) * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long rows = (long long)g.B * g.heads * g.nt_cap;
+  const long long blocks = (rows + TOPK_WARPS - 1) / TOPK_WARPS;
+  if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
+  topk_kernel<<<(unsigned)blocks, TOPK_WARPS * 32, smem, s>>>(g, scores, k_cap, idx, mask);
+  return cudaGetLastError();
+}
+
+}  // namespace veda

@@ -1,0 +1,134 @@
+"""One Veda attention layer on the device: the C-ABI calls of the hot path in
+order, over buffers allocated once.
+
+    permute(Q, K, V) -> TripPool(Qp, Kp) -> tile scores -> top-k mask
+      -> tile-skipping sparse attention -> inverse permute
+    (+ distillation rows: full-attention tile map on selected heads and query
+       tiles, row-wise KL against the predicted scores)
+
+Only marshalling and buffer management live here; every step is a libveda
+kernel launch.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+from . import (Layer, veda_full_attn_tilemax, veda_permute, veda_sparse_attn, veda_tile_scores,
+               veda_tile_scores_ws_bytes, veda_topk_mask, veda_trippool)
+
+
+def k_from_keep(keep: float, nt: int) -> int:
+    """Kept key tiles per query tile: round-half-up of keep*nt, at least 1."""
+    return max(1, int(math.floor(keep * nt + 0.5)))
+
+
+@dataclass
+class MapRequest:
+    heads: List[int]                 # heads whose tile map is built
+    rows: Optional[torch.Tensor]     # device int32 [len(heads), n_rows] or None (tiles 0..n_rows-1)
+    n_rows: int
+
+
+class VedaLayer:
+    STAGES = ("permute_q", "permute_k", "permute_v", "trippool_q", "trippool_k", "tile_scores", "topk",
+              "sparse_attn", "unpermute", "tilemap_kl")
+
+    def __init__(self, layer: Layer, keep: Optional[float], weights: Dict[str, torch.Tensor], score_scale: float,
+                 device, k: Optional[Sequence[int]] = None, maps: Optional[MapRequest] = None):
+        self.L = layer
+        self.device = device
+        B, Hh, d = layer.B, layer.heads, layer.d
+        self.k = list(k) if k is not None else [k_from_keep(keep, nt) for nt in layer.nt]
+        self.k_cap = max(self.k)
+        self.hidden = int(weights["w1q"].shape[-1])
+        self.out_dim = int(weights["w2q"].shape[-1])
+        self.w = weights
+        self.score_scale = float(score_scale)
+        self.attn_scale = 1.0 / math.sqrt(d)
+        n_cap, nt_cap = layer.n_cap, layer.nt_cap
+        bf = dict(dtype=torch.bfloat16, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.qp = torch.empty((B, Hh, n_cap, d), **bf)
+        self.kp = torch.empty_like(self.qp)
+        self.vp = torch.empty_like(self.qp)
+        self.op = torch.empty_like(self.qp)
+        self.dq = torch.empty((B, Hh, nt_cap, 3 * d), **f32)
+        self.dk = torch.empty_like(self.dq)
+        self.scores = torch.empty((B, Hh, nt_cap, nt_cap), **f32)
+        self.emb_ws = torch.empty(veda_tile_scores_ws_bytes(layer, self.out_dim) // 4, **f32)
+        self.idx = torch.empty((B, Hh, nt_cap, self.k_cap), dtype=torch.int32, device=device)
+        self.mask = torch.empty((B, Hh, nt_cap, nt_cap), dtype=torch.uint8, device=device)
+        self.perm = torch.empty((Hh, n_cap), dtype=torch.int32, device=device)
+        self.o = torch.empty((B, layer.N, Hh, d), **bf)
+        self.maps = maps
+        if maps is not None:
+            nh = len(maps.heads)
+            self.tilemap = torch.empty((nh, maps.n_rows, nt_cap), **f32)
+            self.map_lse = torch.empty((nh, maps.n_rows, layer.tile), **f32)
+            self.kl_rows = torch.empty((nh, maps.n_rows), **f32)
+            self.kl_out = torch.zeros(4, **f32)
+
+    def effective_flops(self, idx_host=None) -> float:
+        """4*d*sum of kept valid (query, key) token pairs over all heads, from
+        the tile lengths (host arithmetic on the layout)."""
+        L = self.L
+        total = 0
+        for h in range(L.heads):
+            pt, ph, pw = L.tilings[h]
+            nt = L.nt[h]
+            tps = (L.H // ph) * (L.W // pw)
+            lens = [min(pt, L.T - (t // tps) * pt) * ph * pw for t in range(nt)]
+            if idx_host is None:
+                # every query tile keeps k tiles; exact count needs the lists
+                raise ValueError("pass the index lists")
+            for b in range(L.B):
+                rows = idx_host[b, h, :nt, : self.k[h]]
+                key_tok = torch.tensor(lens, dtype=torch.int64)[rows.long()].sum(dim=1)
+                total += int((torch.tensor(lens, dtype=torch.int64) * key_tok).sum())
+        return 4.0 * L.d * total
+
+    # -- the hot path -------------------------------------------------------
+    def front(self, q, k, v, stream=None):
+        L = self.L
+        veda_permute(L, q, self.qp, self.perm, stream=stream)
+        veda_permute(L, k, self.kp, stream=stream)
+        veda_permute(L, v, self.vp, stream=stream)
+        veda_trippool(L, self.qp, self.dq, stream=stream)
+        veda_trippool(L, self.kp, self.dk, stream=stream)
+        w = self.w
+        veda_tile_scores(L, self.dq, self.dk, w["w1q"], w["b1q"], w["w2q"], w["b2q"], w["w1k"], w["b1k"], w["w2k"],
+                         w["b2k"], self.hidden, self.out_dim, self.score_scale, self.scores, self.emb_ws,
+                         stream=stream)
+        veda_topk_mask(L, self.scores, self.k, self.k_cap, self.idx, self.mask, stream=stream)
+
+    def attend(self, stream=None):
+        veda_sparse_attn(self.L, self.qp, self.kp, self.vp, self.idx, self.k, self.k_cap, self.attn_scale, self.op,
+                         stream=stream)
+        veda_permute(self.L, self.o, self.op, inverse=True, stream=stream)
+
+    def distill(self, stream=None):
+        if self.maps is None:
+            return
+        m = self.maps
+        veda_full_attn_tilemax(self.L, self.qp, self.kp, m.heads, m.rows, m.n_rows, self.attn_scale, self.tilemap,
+                               self.map_lse, self.scores, self.kl_rows, self.kl_out, stream=stream)
+
+    def forward(self, q, k, v, stream=None):
+        self.front(q, k, v, stream)
+        self.attend(stream)
+        self.distill(stream)
+        return self.o
+
+    def dense(self, out: torch.Tensor, stream=None):
+        """Same kernel with every tile kept (the library's own dense path)."""
+        veda_sparse_attn(self.L, self.qp, self.kp, self.vp, None, None, 0, self.attn_scale, out, stream=stream)
+
+
+def device_weights(np_weights, device) -> Dict[str, torch.Tensor]:
+    """The same per-head MLP for query and key descriptors (w1, b1, w2, b2)."""
+    w1, b1, w2, b2 = (torch.from_numpy(a).to(device) for a in np_weights)
+    return {"w1q": w1, "b1q": b1, "w2q": w2, "b2q": b2, "w1k": w1, "b1k": b1, "w2k": w2, "b2k": b2}

@@ -1,0 +1,164 @@
+/*
+ * veda.h -- C ABI of libveda.so: the per-layer hot path of Veda's distilled
+ * tile-skipping sparse attention on NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "Technical Summary: Veda - Scalable Video Diffusion
+ * via Distilled Sparse Attention" (gist.science, arXiv 2605.30325), cited as
+ * "Veda summary" with its section. The pages name the steps; layouts, tie
+ * rules and padding are this library's readings, stated at each call.
+ *
+ * Conventions for every call
+ *   - Memory: the caller owns every buffer; the library allocates no device
+ *     memory. Device pointers must be 16-byte aligned.
+ *   - Asynchrony: every call only enqueues kernels on `stream` and returns;
+ *     nothing synchronises except veda_check_status.
+ *   - Errors: argument errors are detected on the host before any launch and
+ *     return VEDA_ERR_INVALID_ARG / VEDA_ERR_UNSUPPORTED with a message in
+ *     veda_last_error() (thread-local). Launch failures return VEDA_ERR_CUDA.
+ *     Kernels never trap: a device-side error (a wait that exceeded its time
+ *     limit, an index outside its range) is written to layer->dev_status and
+ *     read back by veda_check_status.
+ *   - Layouts (row-major, contiguous):
+ *       original tokens  x   [B, N, heads, d] bf16, N = T*H*W,
+ *                            token n = (t*H + y)*W + x
+ *       permuted tokens  xp  [B, heads, n_cap, d] bf16 (per-head tile order)
+ *       descriptors      desc[B, heads, nt_cap, 3d] fp32 ([avg | max | min])
+ *       tile scores          [B, heads, nt_cap, nt_cap] fp32
+ *       key-tile lists   idx [B, heads, nt_cap, k_cap] int32 (ascending, -1 pad)
+ *       tile mask        mask[B, heads, nt_cap, nt_cap] uint8 (0/1)
+ *     Rows/columns of a head beyond its own tile count (nt_h <= i < nt_cap)
+ *     and padding slots are written as zeros (-1 in idx).
+ */
+#ifndef VEDA_H
+#define VEDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum {
+  VEDA_OK = 0,
+  VEDA_ERR_INVALID_ARG = -1,  /* bad sizes, pointers, tilings (host check) */
+  VEDA_ERR_UNSUPPORTED = -2,  /* valid but outside this build's limits      */
+  VEDA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed          */
+  VEDA_ERR_TIMEOUT = -4,      /* device: a pipeline wait exceeded its limit */
+  VEDA_ERR_BAD_INDEX = -5     /* device: a tile index outside [0, nt_h)     */
+} veda_status;
+
+/* A head's tiling pi_{l,h} = (p_t, p_h, p_w): a factorisation of the tile
+ * size into time, height and width extents (Veda summary 2.2). */
+typedef struct {
+  int32_t pt, ph, pw;
+} veda_tiling;
+
+/* One attention layer's geometry.
+ *   B, heads   batch and head count (heads <= 128)
+ *   d          head dimension, 64 or 128
+ *   T, H, W    latent token grid (N = T*H*W tokens)
+ *   tile       tokens per tile, 64 or 128; tilings[h].pt*ph*pw == tile
+ *   tilings    HOST array [heads], read during each call only
+ *   dev_status DEVICE int32 owned by the caller, zero before first use;
+ *              kernels store a veda_status code here instead of trapping.
+ * Padding (a reading; the pages give no rule): p_h | H and p_w | W are
+ * required; T is padded at its end to a multiple of p_t. Tiles are numbered
+ * row-major over (t/p_t, y/p_h, x/p_w) and tokens inside a tile row-major
+ * over (t%p_t, y%p_h, x%p_w), so each tile's valid tokens are a prefix of
+ * length min(p_t, T - t0)*p_h*p_w. */
+typedef struct {
+  int32_t B, heads, d, T, H, W, tile;
+  const veda_tiling* tilings;
+  int32_t* dev_status;
+} veda_layer;
+
+/* Host-only geometry of a layer (no CUDA call). Writes nt[h] (tiles of head
+ * h), n_pad[h] = nt[h]*tile, *n_cap = max n_pad, *nt_cap = max nt. Any output
+ * pointer may be NULL. Returns VEDA_ERR_INVALID_ARG for a bad tiling. */
+int veda_layout(const veda_layer* L, int32_t* nt, int32_t* n_pad, int32_t* n_cap,
+                int32_t* nt_cap);
+
+/* Head-aware tiling permutation (Veda summary 2.2, Head-Aware Tiling).
+ * inverse = 0: x [B,N,heads,d] -> xp [B,heads,n_cap,d]; slot s of head h
+ *   receives token perm_h[s]; padding slots are zero. If `perm` is not NULL
+ *   it receives the index map [heads, n_cap] int32 (original token, or -1).
+ * inverse = 1: xp -> x, the inverse gather; padding rows are dropped.
+ *   `perm` is ignored. */
+int veda_permute(const veda_layer* L, const void* x, void* xp, int32_t* perm,
+                 int inverse, cudaStream_t stream);
+
+/* TripPool descriptors (Veda summary 2.1, Statistic-Aware Estimator): for
+ * each tile and channel, [mean | max | min] over the tile's valid tokens.
+ * xp [B,heads,n_cap,d] bf16 -> desc [B,heads,nt_cap,3d] fp32. */
+int veda_trippool(const veda_layer* L, const void* xp, float* desc, cudaStream_t stream);
+
+/* Head-specific MLP estimator and tile scores (Veda summary 2.1,
+ * Head-Specific Projections): per head h,
+ *   q_i = W2q^T GELU(W1q^T dq_i + b1q) + b2q,  k_j likewise with the k weights,
+ *   scores[i, j] = scale * q_i . k_j          (i, j < nt_h), fp32 FFMA.
+ * GELU is the exact erf form. Weights fp32: w1 [heads, 3d, hidden],
+ * b1 [heads, hidden], w2 [heads, hidden, out_dim], b2 [heads, out_dim];
+ * hidden <= 256, out_dim <= 128 and a multiple of 4. emb_ws is caller scratch
+ * of veda_tile_scores_ws_bytes() bytes (the q and k embeddings). */
+int veda_tile_scores(const veda_layer* L, const float* dq, const float* dk,
+                     const float* w1q, const float* b1q, const float* w2q, const float* b2q,
+                     const float* w1k, const float* b1k, const float* w2k, const float* b2k,
+                     int32_t hidden, int32_t out_dim, float scale, float* scores,
+                     float* emb_ws, cudaStream_t stream);
+size_t veda_tile_scores_ws_bytes(const veda_layer* L, int32_t out_dim);
+
+/* Top-k key tiles per query tile (Veda summary 2.1 and 4: only the highest
+ * scoring key tiles are kept). k: HOST array [heads], 1 <= k[h] <= nt_h,
+ * k[h] <= k_cap. Ranking is on the fp32 value; exact ties (and -0.0 vs +0.0)
+ * go to the lower tile index. idx rows are ascending and -1 padded to k_cap;
+ * `mask` (may be NULL) is the dense 0/1 form. */
+int veda_topk_mask(const veda_layer* L, const float* scores, const int32_t* k, int32_t k_cap,
+                   int32_t* idx, uint8_t* mask, cudaStream_t stream);
+
+/* Tile-skipping sparse attention (Veda summary 2.3): for each query row i of
+ * query tile a, O_i = sum_j softmax_j(scale * q_i . k_j) v_j over the valid
+ * keys j of the key tiles idx[a, 0..k[h]) only; the softmax is renormalised
+ * over those keys and the other tiles are never read. idx == NULL runs the
+ * dense path (every tile kept; k and k_cap ignored). qp/kp/vp/op are
+ * [B,heads,n_cap,d] bf16; lse (may be NULL) [B,heads,n_cap] fp32 receives
+ * the natural-log softmax normaliser. Padding rows of op are zero.
+ * Tensor cores: tcgen05.mma (bf16 in, fp32 accumulate in TMEM); K/V tiles
+ * arrive by TMA. */
+int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const void* vp,
+                     const int32_t* idx, const int32_t* k, int32_t k_cap, float scale,
+                     void* op, float* lse, cudaStream_t stream);
+
+/* Oracle tile map and distillation loss (Veda summary 2.1, Target
+ * Construction and Optimization; 2.3, Training Efficiency): for the selected
+ * heads heads_sel[0..n_heads_sel) (HOST array) and query tiles
+ * qtile_rows [n_heads_sel, n_rows] (DEVICE int32; NULL = tiles 0..n_rows-1),
+ *   pass 1: lse_i = log sum_j exp(scale q_i . k_j) over all valid keys;
+ *   pass 2: tilemap[s, r, b] = max over valid rows i of the tile and valid
+ *           keys j of key tile b of exp(scale q_i . k_j - lse_i),
+ * i.e. max-pooling of the full softmax attention matrix over the tile region.
+ * tilemap [n_heads_sel, n_rows, nt_cap] fp32 (zero beyond nt_h); lse (may be
+ * NULL) [n_heads_sel, n_rows, tile] fp32. If `scores` (the [B=1 batch slice
+ * of] veda_tile_scores output) is not NULL, kl_rows [n_heads_sel, n_rows]
+ * receives KL(t || softmax(scores row)) with t the tile-map row normalised to
+ * sum 1, and *kl_out (device fp32) their mean over rows, then heads.
+ * Only B == 1 layers are accepted. */
+int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp,
+                           const int32_t* heads_sel, int32_t n_heads_sel,
+                           const int32_t* qtile_rows, int32_t n_rows, float scale,
+                           float* tilemap, float* lse, const float* scores,
+                           float* kl_rows, float* kl_out, cudaStream_t stream);
+
+/* Synchronises `stream`, returns the first device-side status recorded in
+ * L->dev_status (VEDA_OK if none) and clears it. */
+int veda_check_status(const veda_layer* L, cudaStream_t stream);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* veda_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VEDA_H */

@@ -1,0 +1,95 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/veda.h declares, computes layouts on the host and rejects bad
+arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_24_b200 as V
+import synth
+from oracle import veda_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "veda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(veda_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert "veda_sparse_attn" in names and len(names) >= 10
+    lib = ctypes.CDLL(V.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(V.EXPORTED)
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
+def test_layout_matches_oracle(idx):
+    w = synth.config(idx)
+    L = V.Layer(w.B, w.heads, w.d, w.T, w.H, w.W, w.tile, w.tilings)
+    lays = [O.head_layout(w.T, w.H, w.W, t) for t in w.tilings]
+    assert L.nt == [l["nt"] for l in lays]
+    assert L.n_pad == [l["n_pad"] for l in lays]
+    assert L.n_cap == max(l["n_pad"] for l in lays)
+    assert L.nt_cap == max(l["nt"] for l in lays)
+
+
+def test_sweep_layouts_have_no_padding():
+    for n in synth.SWEEP_TOKENS:
+        w = synth.sweep(n, 0.1)
+        L = V.Layer(w.B, w.heads, w.d, w.T, w.H, w.W, w.tile, w.tilings)
+        assert all(p == w.N for p in L.n_pad)
+
+
+@pytest.mark.parametrize("tilings,msg", [
+    ([(2, 8, 4)], "factorise"),
+    ([(1, 8, 16)], "divide"),     # W=8 not divisible by 16
+    ([(0, 8, 16)], "non-positive"),
+])
+def test_bad_tilings_rejected(tilings, msg):
+    with pytest.raises(V.VedaError) as e:
+        V.Layer(1, 1, 128, 4, 8, 8, 128, tilings)
+    assert e.value.code == V.VEDA_ERR_INVALID_ARG and msg in str(e.value)
+
+
+def test_unsupported_sizes_rejected():
+    with pytest.raises(V.VedaError) as e:
+        V.Layer(1, 1, 96, 4, 8, 8, 128, [(2, 8, 8)])
+    assert e.value.code == V.VEDA_ERR_UNSUPPORTED
+    with pytest.raises(V.VedaError) as e:
+        V.Layer(1, 1, 128, 4, 8, 8, 32, [(1, 4, 8)])
+    assert e.value.code == V.VEDA_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch():
+    L = V.Layer(1, 2, 64, 4, 8, 8, 64, [(1, 8, 8), (4, 4, 4)])
+    lib = V._lib
+    rc = lib.veda_permute(L.ref, None, None, None, 0, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "NULL" in V.veda_last_error()
+    rc = lib.veda_permute(L.ref, ctypes.c_void_p(0x1008), ctypes.c_void_p(0x2000), None, 0, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "aligned" in V.veda_last_error()
+    k = (ctypes.c_int32 * 2)(5, 1)      # k > nt for head 0
+    rc = lib.veda_topk_mask(L.ref, ctypes.c_void_p(0x1000), k, 8, ctypes.c_void_p(0x2000), None, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "k=5" in V.veda_last_error()
+    rc = lib.veda_sparse_attn(L.ref, *[ctypes.c_void_p(0x1000)] * 3, None, None, 0, ctypes.c_float(-1.0),
+                              ctypes.c_void_p(0x1000), None, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "scale" in V.veda_last_error()
+    sel = (ctypes.c_int32 * 1)(7)
+    rc = lib.veda_full_attn_tilemax(L.ref, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1000), sel, 1, None, 1,
+                                    ctypes.c_float(0.1), ctypes.c_void_p(0x1000), None, None, None, None, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "heads_sel" in V.veda_last_error()
+    rc = lib.veda_check_status(None, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG
+
+
+def test_tile_scores_workspace_size():
+    w = synth.config(3)
+    L = V.Layer(w.B, w.heads, w.d, w.T, w.H, w.W, w.tile, w.tilings)
+    assert V.veda_tile_scores_ws_bytes(L, 64) == 2 * 24 * 1200 * 64 * 4

@@ -1,0 +1,325 @@
+"""GPU parity: every libveda kernel against the fp64 oracle on the same seeded
+inputs, each stage fed the same upstream values as the oracle (top-k gets
+the oracle's fp32 scores, attention gets the oracle's index lists).
+
+Tolerances (from the method's precision):
+  permutation, top-k indices and mask: bit-exact;
+  TripPool: max/min exact, mean within 1e-6 relative (fp32 sum of bf16);
+  tile scores, tile map, KL: per row max|gpu-oracle| <= 1e-3 * max|oracle|;
+  attention output (bf16 in, bf16 out): max abs <= 2e-2, mean abs <= 2e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_24_b200 as V
+import synth
+from oracle import veda_oracle as O
+from tests.helpers import f64, oracle_geometry, oracle_k, small_workloads
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+WL = small_workloads()
+
+
+def _layer(w):
+    return V.Layer(w.B, w.heads, w.d, w.T, w.H, w.W, w.tile, w.tilings, device=DEV)
+
+
+def _inputs(w):
+    return [t.to(DEV) for t in synth.qkv(w, "cpu")]
+
+
+def _permuted(L, w, x):
+    xp = torch.empty((w.B, w.heads, L.n_cap, w.d), dtype=torch.bfloat16, device=DEV)
+    perm = torch.empty((w.heads, L.n_cap), dtype=torch.int32, device=DEV)
+    V.veda_permute(L, x, xp, perm)
+    return xp, perm
+
+
+def _check_attention(out, lse, ref, lens, tile, tol_max=2e-2, tol_mean=2e-3):
+    errs = []
+    for a, (oa, la) in ref.items():
+        got = out[a * tile: a * tile + lens[a]]
+        errs.append(np.abs(got - oa))
+        np.testing.assert_allclose(lse[a * tile: a * tile + lens[a]], la, rtol=1e-3, atol=1e-3)
+    e = np.concatenate([x.ravel() for x in errs])
+    assert e.max() <= tol_max, e.max()
+    assert e.mean() <= tol_mean, e.mean()
+
+
+def _row_rel(got, want, tol=1e-3, floor=1e-30):
+    for g, w_ in zip(np.atleast_2d(got), np.atleast_2d(want)):
+        scale = max(np.abs(w_).max(), floor)
+        assert np.abs(g - w_).max() <= tol * scale, (np.abs(g - w_).max(), scale)
+
+
+# ------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("name", list(WL))
+def test_permute_bit_exact_and_round_trip(name):
+    w = WL[name]
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    assert (L.n_cap, L.nt_cap) == (n_cap, nt_cap)
+    q, k, v = _inputs(w)
+    qp, perm = _permuted(L, w, q)
+    pg = perm.cpu().numpy()
+    for h in range(w.heads):
+        assert np.array_equal(pg[h, :len(perms[h])], perms[h])
+        assert (pg[h, len(perms[h]):] == -1).all()
+    want = O.permute(f64(q), perms, n_cap)
+    assert np.array_equal(f64(qp), want)
+    back = torch.empty_like(q)
+    V.veda_permute(L, back, qp, inverse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(back, q)
+    V.veda_check_status(L)
+
+
+# ---------------------------------------------------------------- TripPool
+
+@pytest.mark.parametrize("name", list(WL))
+def test_trippool(name):
+    w = WL[name]
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, _, _ = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    desc = torch.empty((w.B, w.heads, nt_cap, 3 * w.d), dtype=torch.float32, device=DEV)
+    V.veda_trippool(L, qp, desc)
+    got = desc.cpu().double().numpy()
+    xp = f64(qp)
+    d = w.d
+    for b in range(w.B):
+        for h in range(w.heads):
+            ref = O.trippool(xp[b, h], lays[h]["lens"], w.tile)
+            nt = lays[h]["nt"]
+            np.testing.assert_allclose(got[b, h, :nt, :d], ref[:, :d], rtol=1e-6, atol=1e-6)
+            assert np.array_equal(got[b, h, :nt, d:], ref[:, d:])
+            assert not got[b, h, nt:].any()
+
+
+# ------------------------------------------------------------- tile scores
+
+@pytest.mark.parametrize("name", list(WL))
+def test_tile_scores(name):
+    w = WL[name]
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    rng = np.random.default_rng(5)
+    dq = rng.standard_normal((w.B, w.heads, nt_cap, 3 * w.d)).astype(np.float32)
+    dk = rng.standard_normal((w.B, w.heads, nt_cap, 3 * w.d)).astype(np.float32)
+    w1, b1, w2, b2 = synth.mlp_weights(w)
+    b1 = rng.standard_normal(b1.shape).astype(np.float32) * 0.1   # exercise the biases
+    b2 = rng.standard_normal(b2.shape).astype(np.float32) * 0.1
+    w1k = synth.mlp_weights(synth.custom("k", 1, w.heads, w.d, 1, 1, 1, 64, [(1, 1, 64)] * w.heads, 1, 99))[0]
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    scores = torch.empty((w.B, w.heads, nt_cap, nt_cap), dtype=torch.float32, device=DEV)
+    ws = torch.empty(V.veda_tile_scores_ws_bytes(L, 64) // 4, dtype=torch.float32, device=DEV)
+    V.veda_tile_scores(L, T(dq), T(dk), T(w1), T(b1), T(w2), T(b2), T(w1k), T(b1), T(w2), T(b2), 128, 64,
+                       synth.SCORE_SCALE, scores, ws)
+    got = scores.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt = lays[h]["nt"]
+            ref = O.tile_scores(dq[b, h, :nt].astype(np.float64), dk[b, h, :nt].astype(np.float64), w1[h], b1[h],
+                                w2[h], b2[h], w1k[h], b1[h], w2[h], b2[h], synth.SCORE_SCALE)
+            _row_rel(got[b, h, :nt, :nt], ref)
+            assert not got[b, h, nt:].any() and not got[b, h, :, nt:].any()
+
+
+# -------------------------------------------------------------------- top-k
+
+def _topk_case(w, scores_np, k):
+    L = _layer(w)
+    nt_cap = L.nt_cap
+    k_cap = max(k) + 3
+    idx = torch.empty((w.B, w.heads, nt_cap, k_cap), dtype=torch.int32, device=DEV)
+    mask = torch.empty((w.B, w.heads, nt_cap, nt_cap), dtype=torch.uint8, device=DEV)
+    V.veda_topk_mask(L, torch.from_numpy(scores_np).to(DEV), k, k_cap, idx, mask)
+    gi, gm = idx.cpu().numpy(), mask.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt = L.nt[h]
+            ri, rm = O.topk_rows(scores_np[b, h, :nt, :nt], k[h], k_cap)
+            assert np.array_equal(gi[b, h, :nt], ri)
+            assert np.array_equal(gm[b, h, :nt, :nt], rm)
+            assert (gi[b, h, nt:] == -1).all() and not gm[b, h, nt:].any() and not gm[b, h, :, nt:].any()
+
+
+@pytest.mark.parametrize("name", list(WL))
+@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "signed-zero"])
+def test_topk_bit_exact(name, kind):
+    w = WL[name]
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    rng = np.random.default_rng(6)
+    s = rng.standard_normal((w.B, w.heads, nt_cap, nt_cap)).astype(np.float32)
+    if kind == "ties":
+        s = np.round(s * 2) / 2
+    elif kind == "zeros":
+        s[:] = 0
+    elif kind == "signed-zero":
+        s = np.where(rng.random(s.shape) < 0.5, np.float32(-0.0), np.float32(0.0)).astype(np.float32)
+        s[..., ::3] = 1.0
+    ks = oracle_k(w, lays)
+    _topk_case(w, s, ks)
+    _topk_case(w, s, [1] * w.heads)
+    _topk_case(w, s, [l["nt"] for l in lays])
+
+
+def test_topk_large_rows():
+    w = synth.sweep(261120, 0.03)      # 2040 tiles per row
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    rng = np.random.default_rng(7)
+    s = (rng.standard_normal((1, w.heads, nt_cap, nt_cap)) * 3).astype(np.float32)
+    s = np.round(s * 64) / 64                              # frequent ties
+    _topk_case(w, s, oracle_k(w, lays))
+
+
+# --------------------------------------------------------- sparse attention
+
+def _attention_case(w, k_override=None, dense=False, random_lists=True):
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, k, v = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    kp, _ = _permuted(L, w, k)
+    vp, _ = _permuted(L, w, v)
+    ks = k_override or oracle_k(w, lays)
+    k_cap = max(ks)
+    idx = np.full((w.B, w.heads, nt_cap, k_cap), -1, np.int32)
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt = lays[h]["nt"]
+            idx[b, h, :nt] = synth.random_index_lists(nt, nt, ks[h], k_cap, seed=100 * b + h + w.seed)
+    op = torch.empty_like(qp)
+    lse = torch.empty((w.B, w.heads, n_cap), dtype=torch.float32, device=DEV)
+    scale = 1 / math.sqrt(w.d)
+    if dense:
+        V.veda_sparse_attn(L, qp, kp, vp, None, None, 0, scale, op, lse)
+    else:
+        V.veda_sparse_attn(L, qp, kp, vp, torch.from_numpy(idx).to(DEV), ks, k_cap, scale, op, lse)
+    V.veda_check_status(L)
+    go, gl = f64(op), lse.cpu().double().numpy()
+    xq, xk, xv = f64(qp), f64(kp), f64(vp)
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt, lens = lays[h]["nt"], lays[h]["lens"]
+            ih = np.tile(np.arange(nt), (nt, 1)) if dense else idx[b, h, :nt]
+            kk = nt if dense else ks[h]
+            ref = O.sparse_attention(xq[b, h], xk[b, h], xv[b, h], ih, kk, lens, w.tile, scale)
+            _check_attention(go[b, h], gl[b, h], ref, lens, w.tile)
+            # padding rows and tiles beyond nt are zero
+            for a in range(nt):
+                assert not go[b, h, a * w.tile + lens[a]:(a + 1) * w.tile].any()
+            assert not go[b, h, nt * w.tile:].any()
+
+
+@pytest.mark.parametrize("name", list(WL))
+def test_sparse_attention_random_lists(name):
+    _attention_case(WL[name])
+
+
+@pytest.mark.parametrize("name", list(WL))
+def test_sparse_attention_dense_path(name):
+    _attention_case(WL[name], dense=True)
+
+
+@pytest.mark.parametrize("name", ["ragged-d128-t128", "odd-d128-t64"])
+def test_sparse_attention_k1_and_keep_all(name):
+    w = WL[name]
+    lays, _, _, _ = oracle_geometry(w)
+    _attention_case(w, k_override=[1] * w.heads)
+    _attention_case(w, k_override=[l["nt"] for l in lays])
+
+
+def test_sparse_attention_deterministic():
+    w = WL["ragged-d128-t128"]
+    L = _layer(w)
+    q, k, v = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    kp, _ = _permuted(L, w, k)
+    vp, _ = _permuted(L, w, v)
+    outs = []
+    for _ in range(2):
+        op = torch.empty_like(qp)
+        V.veda_sparse_attn(L, qp, kp, vp, None, None, 0, 0.1, op)
+        outs.append(op)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_sparse_attention_bad_index_reported():
+    w = WL["ragged-d128-t128"]
+    L = _layer(w)
+    q, k, v = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    idx = torch.zeros((1, w.heads, L.nt_cap, 2), dtype=torch.int32, device=DEV)
+    idx[0, 1, 0, 1] = 10_000
+    op = torch.empty_like(qp)
+    V.veda_sparse_attn(L, qp, qp, qp, idx, [2] * w.heads, 2, 0.1, op)
+    with pytest.raises(V.VedaError) as e:
+        V.veda_check_status(L)
+    assert e.value.code == V.VEDA_ERR_BAD_INDEX
+    V.veda_check_status(L)      # cleared
+
+
+# ----------------------------------------------------- tile map, lse and KL
+
+@pytest.mark.parametrize("name", list(WL))
+def test_tilemap_lse_kl(name):
+    w = WL[name]
+    if w.B != 1:
+        pytest.skip("tile map is defined for B == 1 layers")
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, k, _ = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    kp, _ = _permuted(L, w, k)
+    heads = list(range(w.heads))
+    n_rows = min(l["nt"] for l in lays)
+    rows = np.stack([np.sort(np.random.default_rng(h).choice(lays[h]["nt"], n_rows, replace=False))
+                     for h in heads]).astype(np.int32)
+    rng = np.random.default_rng(8)
+    scores = rng.standard_normal((1, w.heads, nt_cap, nt_cap)).astype(np.float32)
+    tm = torch.empty((len(heads), n_rows, nt_cap), dtype=torch.float32, device=DEV)
+    lse = torch.empty((len(heads), n_rows, w.tile), dtype=torch.float32, device=DEV)
+    klr = torch.empty((len(heads), n_rows), dtype=torch.float32, device=DEV)
+    klo = torch.empty(4, dtype=torch.float32, device=DEV)
+    scale = 1 / math.sqrt(w.d)
+    V.veda_full_attn_tilemax(L, qp, kp, heads, torch.from_numpy(rows).to(DEV), n_rows, scale, tm, lse,
+                             torch.from_numpy(scores).to(DEV), klr, klo)
+    V.veda_check_status(L)
+    gm, gl, gk = tm.cpu().double().numpy(), lse.cpu().double().numpy(), klr.cpu().double().numpy()
+    xq, xk = f64(qp), f64(kp)
+    kl_heads = []
+    for s, h in enumerate(heads):
+        nt, lens = lays[h]["nt"], lays[h]["lens"]
+        M, lse_ref = O.full_tilemap(xq[0, h], xk[0, h], lens, w.tile, scale, rows[s])
+        _row_rel(gm[s, :, :nt], M)
+        assert not gm[s, :, nt:].any()
+        for r, a in enumerate(rows[s]):
+            np.testing.assert_allclose(gl[s, r, :lens[a]], lse_ref[a], rtol=1e-4, atol=1e-4)
+        kl = O.kl_rows(M, scores[0, h, rows[s]][:, :nt])
+        np.testing.assert_allclose(gk[s], kl, rtol=1e-3, atol=1e-5)
+        kl_heads.append(kl.mean())
+    assert float(klo[0]) == pytest.approx(float(np.mean(kl_heads)), rel=1e-3)
+
+
+def test_tilemap_all_rows_default_list():
+    w = WL["cfg0"]
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, k, _ = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    kp, _ = _permuted(L, w, k)
+    tm = torch.empty((2, 4, nt_cap), dtype=torch.float32, device=DEV)
+    V.veda_full_attn_tilemax(L, qp, kp, [1, 0], None, 4, 0.125, tm)
+    gm = tm.cpu().double().numpy()
+    for s, h in enumerate([1, 0]):
+        M, _ = O.full_tilemap(f64(qp)[0, h], f64(kp)[0, h], lays[h]["lens"], w.tile, 0.125)
+        _row_rel(gm[s], M)
