@@ -1,0 +1,458 @@
+"""Benchmark of the Veda tile-skipping attention layer on B200.
+
+A step is one pass of the whole hot path over one synthetic layer (the
+720P-10s-like layer: 40x48x80 latent grid = 153,600 tokens, 24 heads, d=128,
+128-token tiles, 10% of key tiles kept = 90% sparsity):
+  permute Q,K,V -> TripPool Q,K -> MLP tile scores -> top-k mask
+  -> tile-skipping sparse attention -> inverse permute
+  -> full-attention tile map + row-wise KL on 2 heads x 120 query tiles.
+
+`value` is effective attention TFLOP/s over the whole step (4*d*kept valid
+token pairs / step time); the attention kernel alone, the library's dense
+path at sparsity 0 and the roofline of the attention kernel are reported
+beside it. `--impl reference` times the fp64 CPU oracle on a bounded sample
+of the same workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "block-sparse attn ms/layer & effective TFLOP/s at 90% sparsity vs dense path"
+UNIT = "TFLOP/s"
+MAP_ROWS = 120          # query tiles per tile-map head (10% of 1200: sparse supervision)
+KERNELS_PER_STEP = 13   # 3 permute, 2 TripPool, MLP + score GEMM, top-k, attention, unpermute, map, KL rows, KL mean
+
+
+# ------------------------------------------------------------------ ranks
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def dist_init(backend: str, world: int):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Largest value of x over all ranks (the timing rule: the job is as slow
+    as its slowest rank)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def rank_workload_seed(rank: int) -> int:
+    """Each rank processes its own independent layer (weak scaling): same
+    shapes, different seeded activations."""
+    return 7919 * rank
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = float(p[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["bf16_tflops"], d["bf16_tflops_sustained"], d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# --------------------------------------------------------------- our path
+
+def build_layer(w, device, seed_offset=0):
+    import block_sparse_attention_24_b200 as V
+    from block_sparse_attention_24_b200.layer import MapRequest, VedaLayer, device_weights
+    L = V.Layer(w.B, w.heads, w.d, w.T, w.H, w.W, w.tile, w.tilings, device=device)
+    heads = list(w.tilemap_heads)
+    rows = np.stack([synth.sample_rows(L.nt[h], min(MAP_ROWS, L.nt[h]), w.seed + h) for h in heads])
+    maps = MapRequest(heads, torch.from_numpy(rows).to(device), rows.shape[1])
+    layer = VedaLayer(L, w.keep, device_weights(synth.mlp_weights(w), device), synth.SCORE_SCALE, device, maps=maps)
+    q, k, v = synth.qkv(w, device, seed_offset=seed_offset)
+    return V, L, layer, (q, k, v)
+
+
+def kept_pairs(L, layer):
+    """Kept valid (query, key) token pairs and all valid pairs, from the
+    top-k lists and the tile lengths."""
+    idx = layer.idx.cpu()
+    kept = allp = 0
+    for h in range(L.heads):
+        pt, ph, pw = L.tilings[h]
+        tps = (L.H // ph) * (L.W // pw)
+        lens = torch.tensor([min(pt, L.T - (t // tps) * pt) * ph * pw for t in range(L.nt[h])], dtype=torch.int64)
+        for b in range(L.B):
+            rows = idx[b, h, :L.nt[h], :layer.k[h]].long()
+            kept += int((lens * lens[rows].sum(dim=1)).sum())
+            allp += int(lens.sum()) ** 2
+    return kept, allp
+
+
+def run_ours(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init("nccl", world)
+    w = synth.config(args.config, keep=args.keep)
+    V, L, layer, (q, k, v) = build_layer(w, device, seed_offset=rank_workload_seed(rank))
+    stream = torch.cuda.current_stream(device)
+
+    # warm-up
+    for _ in range(args.warmup):
+        layer.forward(q, k, v)
+    torch.cuda.synchronize(device)
+    V.veda_check_status(L)
+    kept, allp = kept_pairs(L, layer)
+    eff_flops = 4.0 * L.d * kept
+    n_stage = len(layer.STAGES)
+
+    # timed region: whole steps, with events around each stage on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for s in range(args.steps):
+            e = ev[s]
+            e[0].record(stream)
+            layer.front(q, k, v)
+            e[1].record(stream)
+            V.veda_sparse_attn(L, layer.qp, layer.kp, layer.vp, layer.idx, layer.k, layer.k_cap, layer.attn_scale,
+                               layer.op)
+            e[2].record(stream)
+            V.veda_permute(L, layer.o, layer.op, inverse=True)
+            e[3].record(stream)
+            layer.distill()
+            e[4].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier()
+    elapsed = t0.elapsed_time(t1) / 1e3
+    elapsed = max_over_ranks(elapsed, device)
+    V.veda_check_status(L)
+    front_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    unperm_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    map_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in ev)
+    clocks = clk.summary()
+
+    # per-stage breakdown of the front end (separate, untimed-for-value pass)
+    stage_ms = stage_breakdown(V, L, layer, q, k, v, stream)
+
+    # dense path (same kernel, every tile kept) on the same permuted tensors
+    dense_out = torch.empty_like(layer.op)
+    layer.dense(dense_out)
+    torch.cuda.synchronize(device)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = args.dense_reps
+    d0.record(stream)
+    for _ in range(reps):
+        layer.dense(dense_out)
+    d1.record(stream)
+    torch.cuda.synchronize(device)
+    dense_ms = d0.elapsed_time(d1) / reps
+    del dense_out
+
+    e2e = run_e2e(V, L, layer, q, k, v, device, eff_flops, args)
+
+    burst, sustained, hbm, src = measured_peaks()
+    attn_tflops = eff_flops / (attn_ms / 1e3) / 1e12
+    step_ms = elapsed / args.steps * 1e3
+    value = world * eff_flops / (elapsed / args.steps) / 1e12
+    traffic = load_traffic()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, layer, L, budget_s=args.cpu_seconds)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "model": "none (one attention layer, synthetic activations)",
+                   "global_batch": w.B * world, "seq_len": w.N, "heads": w.heads, "head_dim": w.d,
+                   "tile": w.tile, "keep": w.keep, "sparsity": round(1 - kept / allp, 4),
+                   "tilemap": {"heads": list(w.tilemap_heads), "query_tiles_per_head": int(layer.maps.n_rows)},
+                   "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (each of Q/K/V is 944 MB)"},
+        "attn_ms": round(attn_ms, 3), "attn_tflops": round(attn_tflops, 1),
+        "attn_frac_of_burst_peak": round(attn_tflops / burst, 4),
+        "dense_ms": round(dense_ms, 3), "speedup_vs_dense": round(dense_ms / attn_ms, 2),
+        "layer_ms": round(front_ms + attn_ms + unperm_ms, 3),
+        "stage_ms": {**stage_ms, "front_end": round(front_ms, 3), "sparse_attn": round(attn_ms, 3),
+                     "unpermute": round(unperm_ms, 3), "tilemap_kl": round(map_ms, 3)},
+        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": sustained, "unit": UNIT,
+                     "frac": round(attn_tflops / sustained, 4), "traffic": traffic,
+                     "kernel": "sparse_attn_kernel<128,128>",
+                     "peak_kind": f"bf16 dense sustained ({src}); burst {burst}"},
+        "e2e": e2e,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def stage_breakdown(V, L, layer, q, k, v, stream):
+    names = ["permute_qkv", "trippool_qk", "tile_scores", "topk"]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+    w = layer.w
+    ev[0].record(stream)
+    V.veda_permute(L, q, layer.qp, layer.perm)
+    V.veda_permute(L, k, layer.kp)
+    V.veda_permute(L, v, layer.vp)
+    ev[1].record(stream)
+    V.veda_trippool(L, layer.qp, layer.dq)
+    V.veda_trippool(L, layer.kp, layer.dk)
+    ev[2].record(stream)
+    V.veda_tile_scores(L, layer.dq, layer.dk, w["w1q"], w["b1q"], w["w2q"], w["b2q"], w["w1k"], w["b1k"], w["w2k"],
+                       w["b2k"], layer.hidden, layer.out_dim, layer.score_scale, layer.scores, layer.emb_ws)
+    ev[3].record(stream)
+    V.veda_topk_mask(L, layer.scores, layer.k, layer.k_cap, layer.idx, layer.mask)
+    ev[4].record(stream)
+    torch.cuda.synchronize()
+    return {n: round(ev[i].elapsed_time(ev[i + 1]), 3) for i, n in enumerate(names)}
+
+
+def run_e2e(V, L, layer, q, k, v, device, eff_flops, args):
+    """Host buffers in, host result out, through the same public calls."""
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(layer.o.shape, dtype=layer.o.dtype).pin_memory()
+    hkl = torch.empty(4, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        layer.forward(dq, dk, dv)
+        ho.copy_(layer.o, non_blocking=True)
+        hkl.copy_(layer.kl_out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.e2e_steps, device)
+    world = dist_env()[0]
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hkl.numel() * hkl.element_size()
+    return {"value": round(world * eff_flops / t / 1e12, 3), "unit": UNIT, "ms_per_step": round(t * 1e3, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+
+def load_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    matches the current kernel (written by hand from an ncu capture)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("sparse_attn_bytes_per_launch")
+    return None
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_attention_sample(w, qp_h, kp_h, vp_h, idx_h, k, lens, budget_s, seed=0):
+    """Runs the oracle's sparse attention tile by tile on seeded query tiles
+    until `budget_s` seconds are used; returns (effective flops, seconds,
+    tiles)."""
+    from oracle import veda_oracle as O
+    nt = len(lens)
+    order = np.random.default_rng(seed).permutation(nt)
+    flops, tiles = 0.0, 0
+    t0 = time.perf_counter()
+    for a in order:
+        O.sparse_attention(qp_h, kp_h, vp_h, idx_h, k, lens, w.tile, 1 / math.sqrt(w.d), rows=[int(a)])
+        flops += 4.0 * w.d * O.effective_pairs(lens, idx_h, k, rows=[int(a)])
+        tiles += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return flops, time.perf_counter() - t0, tiles
+
+
+def cpu_baseline(w, layer, L, budget_s):
+    from oracle import veda_oracle as O
+    h = 0
+    lens = O.head_layout(w.T, w.H, w.W, w.tilings[h])["lens"]
+    f = lambda t: t[0, h].float().cpu().double().numpy()
+    qp, kp, vp = f(layer.qp), f(layer.kp), f(layer.vp)
+    idx = layer.idx[0, h].cpu().numpy()
+    flops, secs, tiles = oracle_attention_sample(w, qp, kp, vp, idx, layer.k[h], lens, budget_s)
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"fp64 NumPy sparse attention, head {h}, {tiles} random query tiles of 1200 "
+                      f"({secs:.1f} s); the front end is not included"}
+
+
+def run_reference(args, world, rank, local):
+    """The fp64 CPU oracle as the reference arm: each step = the oracle's
+    front end for one head (permute, TripPool, MLP scores, top-k) plus its
+    sparse attention on seeded query tiles of that head."""
+    if rank != 0:
+        return
+    from oracle import veda_oracle as O
+    w = synth.config(args.config, keep=args.keep)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    q, k, v = synth.qkv(w, dev)
+    w1, b1, w2, b2 = synth.mlp_weights(w)
+    h = 0
+    tiling = w.tilings[h]
+    lay = O.head_layout(w.T, w.H, w.W, tiling)
+    perm = O.perm_indices(w.T, w.H, w.W, tiling)
+    qh, kh, vh = (t[:, :, h:h + 1].float().cpu().double().numpy() for t in (q, k, v))
+    del q, k, v
+    kk = O.k_from_keep(w.keep, lay["nt"])
+
+    def step(budget):
+        t0 = time.perf_counter()
+        qp, kp, vp = (O.permute(x, [perm], lay["n_pad"])[0, 0] for x in (qh, kh, vh))
+        dq = O.trippool(qp, lay["lens"], w.tile)
+        dk = O.trippool(kp, lay["lens"], w.tile)
+        s = O.tile_scores(dq, dk, w1[h], b1[h], w2[h], b2[h], w1[h], b1[h], w2[h], b2[h], synth.SCORE_SCALE)
+        idx, _ = O.topk_rows(s, kk)
+        front = time.perf_counter() - t0
+        flops, secs, tiles = oracle_attention_sample(w, qp, kp, vp, idx, kk, lay["lens"], budget)
+        return flops, front + secs, tiles
+
+    for _ in range(args.warmup):
+        step(1.0)
+    tot_f = tot_s = 0.0
+    tiles = 0
+    for _ in range(args.steps):
+        f, s_, t = step(args.ref_step_seconds)
+        tot_f += f
+        tot_s += s_
+        tiles += t
+    value = tot_f / tot_s / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "keep": w.keep, "tile": w.tile},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"per step: oracle front end for head {h} + sparse attention on "
+                                   f"~{tiles / max(1, args.steps):.0f} seeded query tiles"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--keep", type=float, default=None)
+    ap.add_argument("--dense-reps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps are required")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()
