@@ -2,7 +2,7 @@
 extension machinery): one object per .cu file under csrc/, linked with the
 static CUDA runtime so the library depends only on the driver at run time.
 
-    python -m block_sparse_attention_24_b200.build [--verbose]
+    python block_sparse_attention_24_b200/build.py [--verbose]
 """
 from __future__ import annotations
 
