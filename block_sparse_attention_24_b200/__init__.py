@@ -26,6 +26,7 @@ VEDA_ERR_TIMEOUT = -4
 VEDA_ERR_BAD_INDEX = -5
 
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
+            "veda_tile_scores_noalloc",
             "veda_topk_mask", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
             "veda_last_error")
 
@@ -38,7 +39,7 @@ class VedaError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(_LIB_PATH):
-        raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m block_sparse_attention_24_b200.build`")
+        raise ImportError(f"{_LIB_PATH} is missing: build it with `python block_sparse_attention_24_b200/build.py`")
     return ctypes.CDLL(_LIB_PATH)
 
 
@@ -63,6 +64,7 @@ _lib.veda_layout.argtypes = [_LP, _P, _P, _P, _P]
 _lib.veda_permute.argtypes = [_LP, _P, _P, _P, ctypes.c_int, _P]
 _lib.veda_trippool.argtypes = [_LP, _P, _P, _P]
 _lib.veda_tile_scores.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _P, _P]
+_lib.veda_tile_scores_noalloc.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _P]
 _lib.veda_tile_scores_ws_bytes.argtypes = [_LP, _I]
 _lib.veda_tile_scores_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_topk_mask.argtypes = [_LP, _P, _P, _I, _P, _P, _P]
@@ -153,6 +155,16 @@ def veda_tile_scores(layer: Layer, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2
                      scale: float, scores: torch.Tensor, emb_ws: torch.Tensor, stream=None):
     _check(_lib.veda_tile_scores(layer.ref, *[_ptr(t) for t in (dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k)],
                                  hidden, out_dim, float(scale), _ptr(scores), _ptr(emb_ws), _stream(stream)))
+
+
+def veda_tile_scores_noalloc(layer: Layer, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden: int,
+                             out_dim: int, scale: float, scores: torch.Tensor, stream=None):
+    """veda_tile_scores for callers that cannot allocate device memory: the
+    embeddings go to a 16 MiB array built into the library (shared by all
+    calls; overlapping calls race)."""
+    _check(_lib.veda_tile_scores_noalloc(layer.ref, *[_ptr(t) for t in (dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k,
+                                                                         b2k)],
+                                         hidden, out_dim, float(scale), _ptr(scores), _stream(stream)))
 
 
 def _host_i32(vals):

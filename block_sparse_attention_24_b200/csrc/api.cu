@@ -286,3 +286,17 @@ int veda_check_status(const veda_layer* L, cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+namespace veda {
+
+// Records a message for veda_last_error() from code outside this file.
+void set_last_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
+}  // namespace veda

@@ -110,6 +110,24 @@ int veda_tile_scores(const veda_layer* L, const float* dq, const float* dk,
                      float* emb_ws, cudaStream_t stream);
 size_t veda_tile_scores_ws_bytes(const veda_layer* L, int32_t out_dim);
 
+/* veda_tile_scores without a scratch argument, for callers that may not
+ * allocate device memory: applications that load this library as a plug-in
+ * and own every byte of device memory in a pre-planned pool, and real-time
+ * loops that must not call an allocator between frames. The pages describe
+ * no such call; it is a deployment variant of the call above with identical
+ * results. The embeddings live in a device array built into the library
+ * (16 MiB, held by every GPU that loads the library until the process
+ * exits); a layer needing more (veda_tile_scores_ws_bytes > 16 MiB) is
+ * rejected with VEDA_ERR_UNSUPPORTED. The first call on each device looks up
+ * that device's copy of the array (make it before any stream capture). All
+ * calls share the array: calls whose kernels may overlap on the GPU race and
+ * must be serialised by the caller. Allocates nothing. */
+int veda_tile_scores_noalloc(const veda_layer* L, const float* dq, const float* dk,
+                             const float* w1q, const float* b1q, const float* w2q, const float* b2q,
+                             const float* w1k, const float* b1k, const float* w2k, const float* b2k,
+                             int32_t hidden, int32_t out_dim, float scale, float* scores,
+                             cudaStream_t stream);
+
 /* Top-k key tiles per query tile (Veda summary 2.1 and 4: only the highest
  * scoring key tiles are kept). k: HOST array [heads], 1 <= k[h] <= nt_h,
  * k[h] <= k_cap. Ranking is on the fp32 value; exact ties (and -0.0 vs +0.0)
