@@ -79,6 +79,15 @@ def rank_workload_seed(rank: int) -> int:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
+    """nvidia-smi sampling (100 ms) of SM clock, power and throttle reasons.
+    Started before the warm-up so its start-up never lands in the timed
+    region; `summary(t0, t1)` keeps only samples taken inside [t0, t1]
+    (host wall clock, as datetime.now())."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
     def __init__(self, index: int):
         self.index = index
         self.proc = None
@@ -86,13 +95,10 @@ class ClockSampler:
 
     def __enter__(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -107,25 +113,31 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, mx, reasons = [], None, set()
+        sm, pw, mx, reasons = [], [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             p = [x.strip() for x in line.split(",")]
-            if len(p) < 9:
+            if len(p) < 10:
                 continue
             try:
-                sm.append(float(p[1]))
-                mx = float(p[2])
+                ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f")
+                clk, mx_, pwr = float(p[2]), float(p[3]), float(p[4])
             except ValueError:
                 continue
-            for n, v in zip(names, p[5:9]):
+            if t0 is not None and not (t0 <= ts <= t1):
+                continue
+            sm.append(clk)
+            pw.append(pwr)
+            mx = mx_
+            for n, v in zip(names, p[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "power_w_median": statistics.median(pw) if pw else None, "samples": len(sm),
+                "period_ms": 100}
 
 
 def measured_peaks():
@@ -174,6 +186,7 @@ def run_ours(args, world, rank, local):
     V, L, layer, (q, k, v) = build_layer(w, device, seed_offset=rank_workload_seed(rank))
     stream = torch.cuda.current_stream(device)
 
+    clk = ClockSampler(local).__enter__()
     # warm-up
     for _ in range(args.warmup):
         layer.forward(q, k, v)
@@ -187,7 +200,8 @@ def run_ours(args, world, rank, local):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize(device)
-    with ClockSampler(local) as clk:
+    if True:
+        host_t0 = datetime.datetime.now()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -205,6 +219,7 @@ def run_ours(args, world, rank, local):
             e[4].record(stream)
         t1.record(stream)
         torch.cuda.synchronize(device)
+        host_t1 = datetime.datetime.now()
     barrier()
     elapsed = t0.elapsed_time(t1) / 1e3
     elapsed = max_over_ranks(elapsed, device)
@@ -213,7 +228,8 @@ def run_ours(args, world, rank, local):
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     unperm_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
     map_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in ev)
-    clocks = clk.summary()
+    clk.__exit__(None, None, None)
+    clocks = clk.summary(host_t0, host_t1)
 
     # per-stage breakdown of the front end (separate, untimed-for-value pass)
     stage_ms = stage_breakdown(V, L, layer, q, k, v, stream)
@@ -434,7 +450,7 @@ def run_reference(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=3)

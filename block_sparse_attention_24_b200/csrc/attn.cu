@@ -1,24 +1,28 @@
 // Tile-skipping sparse attention on sm_100a (Veda summary 2.3, Hardware-
-// Efficient Implementation): each CTA owns 128 query rows of one head and
-// walks only the key/value tiles its query tiles kept; skipped tiles are
-// never loaded.
+// Efficient Implementation), one 128-row query block per CTA: each CTA walks
+// only the key/value tiles its query tiles kept; skipped tiles are never
+// loaded. Used for 64-token tiles; 128-token tiles go to the two-tile kernel
+// in attn_pair.cu.
 //
-// Roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r. Reads S from
-//              TMEM, keeps the running max / sum in fp32, writes P (bf16) to
-//              shared memory, rescales O in TMEM when the max grows by more
-//              than 2^8, and finally normalises O and stores it.
-//   warp 4     producer: TMA loads of Q once and of the selected K and V tiles
-//              into two-stage rings (128B-swizzled).
-//   warp 5     MMA issuer (one thread): S = Q K^T into one of two TMEM
-//              buffers, O += P V into a TMEM accumulator, tcgen05.commit to
-//              mbarriers.
-// Pipeline per key block j: S_j is computed while softmax j-1 runs, PV_j and
-// S_{j+2} are queued as soon as P_j is written.
+// Roles (224 threads):
+//   warps 0-3  softmax: thread r owns query row r = TMEM lane r. Reads a row
+//              of S from TMEM, keeps the running max / sum in fp32, writes P
+//              (bf16 pairs) back into the first half of the same TMEM
+//              columns, rescales O in TMEM when the max grows by more than
+//              2^8, and finally normalises O and stores it.
+//   warp 4     K producer: TMA loads of Q once and of the selected K tiles
+//              into a 3-stage ring (128B-swizzled).
+//   warp 5     MMA issuer (one thread): S = Q K^T (A, B from shared memory)
+//              into one of two TMEM buffers; O += P V with P read from TMEM
+//              and V from shared memory; tcgen05.commit to mbarriers.
+//   warp 6     V producer: TMA loads of the selected V tiles, 3-stage ring.
+// K and V have their own producers so a K load never waits behind a V slot.
+// Per key block j the MMA warp queues PV_j and then S_{j+2} as soon as P_j
+// is in TMEM, so the tensor core works on them while softmax j+1 runs.
 //
 // Tiles of 64 tokens: a CTA still computes 128x128 blocks; its two 64-row
 // query tiles each pair with their own 64-key tile, so only the two diagonal
-// 64x64 blocks of S are used (the others are masked to zero in P).
+// 64x64 blocks of S are used (the others are zero in P).
 //
 // Every mbarrier wait is bounded (VEDA_WAIT_LIMIT_NS); on expiry the CTA
 // records VEDA_ERR_TIMEOUT, drains the copies and MMAs it issued, frees its
@@ -30,21 +34,22 @@ namespace {
 
 constexpr int BM = 128;               // query rows per CTA
 constexpr int BN = 128;               // keys per block
+constexpr int KST = 3, VST = 3;       // K and V ring stages
 constexpr float RESCALE_LOG2 = 8.0f;  // rescale O only when the max grows by > 2^8
-constexpr uint32_t TMEM_COLS = 512;
-constexpr int NUM_THREADS = 192;
+constexpr int POLY_PAIRS = 0x8;       // which of the 4 pairs per 8-key chunk use the FMA-pipe exp2
+constexpr uint32_t TMEM_COLS = 512;   // S0 [0,128), S1 [128,256), O [256, 256+D)
+constexpr int NUM_THREADS = 224;
 
 template <int D>
 struct AttnLayout {
   static constexpr int QB = BM * D * 2;       // Q block bytes (D/64 boxes of 16 KB)
   static constexpr int KB = BN * D * 2;       // K or V block bytes
-  static constexpr int PB = BM * BN * 2;      // P block bytes (2 boxes of 16 KB)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QB;
-  static constexpr int OFF_V = OFF_K + 2 * KB;
-  static constexpr int OFF_P = OFF_V + 2 * KB;
-  static constexpr int OFF_BAR = OFF_P + 2 * PB;
-  static constexpr int NUM_BARS = 16;
+  static constexpr int OFF_V = OFF_K + KST * KB;
+  static constexpr int OFF_BAR = OFF_V + VST * KB;
+  // q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], p_full[2], pv_done[2], drain
+  static constexpr int NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
@@ -58,8 +63,8 @@ struct AttnParams {
   float* lse;
 };
 
-// Tile index of query sub-tile `sub` at key block `j` (clamped into range;
-// an out-of-range entry is reported once).
+// Key tile at block j of an index row (dense path: j itself), clamped into
+// range; an out-of-range entry is reported.
 __device__ __forceinline__ int key_tile(const int32_t* row, int j, int nt, int32_t* status) {
   if (!row) return j;
   int t = __ldg(row + j);
@@ -92,7 +97,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (qb >= n_qb) {  // padding rows of this head: zero output
     for (int i = threadIdx.x; i < BM * D / 8; i += NUM_THREADS) {
       const int r = i / (D / 8);
-      if (qb * BM + r < g.n_cap) reinterpret_cast<uint4*>(prm.op + (row0 + r) * D)[i % (D / 8)] = make_uint4(0, 0, 0, 0);
+      if (qb * BM + r < g.n_cap)
+        reinterpret_cast<uint4*>(prm.op + (row0 + r) * D)[i % (D / 8)] = make_uint4(0, 0, 0, 0);
     }
     if (prm.lse)
       for (int r = threadIdx.x; r < BM; r += NUM_THREADS)
@@ -102,15 +108,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   uint8_t* sQ = smem + Lay::OFF_Q;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* p_full = bars + 11;  // [2]
-  uint64_t* pv_done = bars + 13; // [2]
-  uint64_t* mma_drain = bars + 15;
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* s_full = v_empty + VST;  // [2]
+  uint64_t* p_full = s_full + 2;     // [2], 128 arrivals
+  uint64_t* pv_done = p_full + 2;    // [2]
+  uint64_t* mma_drain = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
 
@@ -124,7 +130,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < Lay::NUM_BARS; ++i) mbar_init(bars + i, (i == 11 || i == 12) ? 128 : 1);  // p_full: 128
+    for (int i = 0; i < Lay::NUM_BARS; ++i) {
+      uint64_t* bar = bars + i;
+      mbar_init(bar, (bar == p_full || bar == p_full + 1) ? 128 : 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -136,46 +145,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == 4 || warp == 6) {
+    // ----------------------------------------------------------- producers
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_expect_tx(q_full, Lay::QB);
+      const bool is_k = warp == 4;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      uint8_t* ring = smem + (is_k ? Lay::OFF_K : Lay::OFF_V);
+      constexpr int ST = KST;  // == VST
+      tma_prefetch_desc(map);
+      if (is_k) {
+        tma_prefetch_desc(&tmQ);
+        mbar_expect_tx(q_full, Lay::QB);
 #pragma unroll
-      for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(sQ + bx * BM * 128, &tmQ, q_full, bx * 64, qb * BM, bh);
-      int kt_issued = 0, vt_issued = 0;
+        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(sQ + bx * BM * 128, &tmQ, q_full, bx * 64, qb * BM, bh);
+      }
+      int issued = 0;
       for (int t = 0; t < n; ++t) {
-        const int s = t & 1;
+        const int st = t % ST;
         int kts[NSUB];
 #pragma unroll
-        for (int u = 0; u < NSUB; ++u) kts[u] = key_tile(lists[u], t, nt, g.dev_status);
-        if (t >= 2 && !mbar_wait(k_empty + s, ((t - 2) >> 1) & 1, abort_flag, g.dev_status)) break;
-        mbar_expect_tx(k_full + s, Lay::KB);
-        uint8_t* dK = smem + Lay::OFF_K + s * Lay::KB;
+        for (int u = 0; u < NSUB; ++u) kts[u] = key_tile(lists[u], t, nt, is_k ? g.dev_status : nullptr);
+        if (t >= ST && !mbar_wait(empty + st, ((t - ST) / ST) & 1, abort_flag, g.dev_status)) break;
+        mbar_expect_tx(full + st, Lay::KB);
+        uint8_t* dst = ring + st * Lay::KB;
 #pragma unroll
         for (int u = 0; u < NSUB; ++u)
 #pragma unroll
           for (int bx = 0; bx < D / 64; ++bx)
-            tma_load_3d(dK + bx * BN * 128 + u * TILE * 128, &tmK, k_full + s, bx * 64, kts[u] * TILE, bh);
-        kt_issued = t + 1;
-        if (t >= 2 && !mbar_wait(v_empty + s, ((t - 2) >> 1) & 1, abort_flag, g.dev_status)) break;
-        mbar_expect_tx(v_full + s, Lay::KB);
-        uint8_t* dV = smem + Lay::OFF_V + s * Lay::KB;
-#pragma unroll
-        for (int u = 0; u < NSUB; ++u)
-#pragma unroll
-          for (int bx = 0; bx < D / 64; ++bx)
-            tma_load_3d(dV + bx * BN * 128 + u * TILE * 128, &tmV, v_full + s, bx * 64, kts[u] * TILE, bh);
-        vt_issued = t + 1;
+            tma_load_3d(dst + bx * BN * 128 + u * TILE * 128, map, full + st, bx * 64, kts[u] * TILE, bh);
+        issued = t + 1;
       }
-      if (*abort_flag) {  // let every copy this CTA started land before exiting
-        mbar_wait_drain(q_full, 0, VEDA_WAIT_LIMIT_NS);
-        for (int t = kt_issued - 2 < 0 ? 0 : kt_issued - 2; t < kt_issued; ++t)
-          mbar_wait_drain(k_full + (t & 1), (t >> 1) & 1, VEDA_WAIT_LIMIT_NS);
-        for (int t = vt_issued - 2 < 0 ? 0 : vt_issued - 2; t < vt_issued; ++t)
-          mbar_wait_drain(v_full + (t & 1), (t >> 1) & 1, VEDA_WAIT_LIMIT_NS);
+      if (*abort_flag) {  // let every copy this warp started land before exiting
+        if (is_k) mbar_wait_drain(q_full, 0, VEDA_WAIT_LIMIT_NS);
+        for (int t = issued - ST < 0 ? 0 : issued - ST; t < issued; ++t)
+          mbar_wait_drain(full + t % ST, (t / ST) & 1, VEDA_WAIT_LIMIT_NS);
       }
     }
   } else if (warp == 5) {
@@ -186,19 +191,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t aQ = smem_u32(sQ);
       const uint32_t aK = smem_u32(smem + Lay::OFF_K);
       const uint32_t aV = smem_u32(smem + Lay::OFF_V);
-      const uint32_t aP = smem_u32(smem + Lay::OFF_P);
       auto issue_s = [&](int t) -> bool {
-        const int s = t & 1;
-        if (!mbar_wait(k_full + s, (t >> 1) & 1, abort_flag, g.dev_status)) return false;
+        const int s = t & 1, st = t % KST;
+        if (!mbar_wait(k_full + st, (t / KST) & 1, abort_flag, g.dev_status)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
           umma_bf16_ss(tmem + s * BN, sdesc_sw128(aQ + off, 16, 1024),
-                       sdesc_sw128(aK + s * Lay::KB + off, 16, 1024), idesc_s, kk > 0);
+                       sdesc_sw128(aK + st * Lay::KB + off, 16, 1024), idesc_s, kk > 0);
         }
         umma_commit(s_full + s);
-        umma_commit(k_empty + s);
+        umma_commit(k_empty + st);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, abort_flag, g.dev_status);
@@ -206,21 +210,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         for (int t = 0; t < 2 && t < n && ok; ++t) ok = issue_s(t);
         for (int j = 0; j < n && ok; ++j) {
-          const int s = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          if (!mbar_wait(p_full + s, ph, abort_flag, g.dev_status)) break;
-          if (!mbar_wait(v_full + s, ph, abort_flag, g.dev_status)) break;
+          const int s = j & 1, sv = j % VST;
+          if (!mbar_wait(p_full + s, (j >> 1) & 1, abort_flag, g.dev_status)) break;
+          if (!mbar_wait(v_full + sv, (j / VST) & 1, abort_flag, g.dev_status)) break;
           tc_fence_after();
+          // P_j sits in the first 64 columns of S buffer s (two bf16 per column)
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-            umma_bf16_ss(tmem + 2 * BN, sdesc_sw128(aP + s * Lay::PB + offp, 16, 1024),
-                         sdesc_sw128(aV + s * Lay::KB + kk * 2048, BN * 128, 1024), idesc_o,
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_bf16_ts(tmem + 2 * BN, tmem + s * BN + kk * 8,
+                         sdesc_sw128(aV + sv * Lay::KB + kk * 2048, BN * 128, 1024), idesc_o,
                          (j > 0 || kk > 0) ? 1u : 0u);
-          }
           umma_commit(pv_done + s);
-          umma_commit(v_empty + s);
-          if (j + 2 < n) ok = issue_s(j + 2);
+          umma_commit(v_empty + sv);
+          if (j + 2 < n) ok = issue_s(j + 2);  // overwrites S buffer s after PV_j has read P_j
         }
       }
       umma_commit(mma_drain);
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool row_valid = a < nt && (r % TILE) < tile_len(hg, g.T, a);
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     const float C = prm.scale_log2;
-    uint8_t* sP = smem + Lay::OFF_P;
+    const uint64_t C2 = f2(C, C);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -246,20 +248,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, ph, abort_flag, g.dev_status))) { ok = false; break; }
       tc_fence_after();
       float sv[TILE];
+      {
+        uint32_t u[TILE];
+        if constexpr (TILE == 128) tmem_ld128(lane_addr + s * BN, u);
+        else tmem_ld64(lane_addr + s * BN + sub * TILE, u);
 #pragma unroll
-      for (int c = 0; c < TILE / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(lane_addr + s * BN + sub * TILE + c * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < TILE; ++e) sv[e] = __uint_as_float(u[e]);
       }
-      float mx = -INFINITY;
-      if (klen == TILE) {
+      const bool full = klen == TILE;
+      if (!full) {  // padded key tile: mask the columns past its valid prefix
 #pragma unroll
-        for (int c = 0; c < TILE; ++c) mx = fmaxf(mx, sv[c]);
-      } else {
+        for (int c = 0; c < TILE; ++c) sv[c] = c < klen ? sv[c] : -INFINITY;
+      }
+      // row max: 8 independent 3-input max chains
+      float mx;
+      {
+        float pm[8];
 #pragma unroll
-        for (int c = 0; c < TILE; ++c) mx = fmaxf(mx, c < klen ? sv[c] : -INFINITY);
+        for (int i = 0; i < 8; ++i) pm[i] = fmaxf(sv[i], sv[i + 8]);
+#pragma unroll
+        for (int c = 16; c < TILE; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], sv[c + i], sv[c + 8 + i]);
+        mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
       }
       const float mx2 = mx * C;
       if (j == 0) {
@@ -268,7 +279,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool need = mx2 > m + RESCALE_LOG2;
         if (__any_sync(0xffffffffu, need)) {
           // O must hold PV_{j-1} before it is rescaled
-          if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, g.dev_status))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
+                                                 g.dev_status))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const float alpha = need ? fast_exp2(m - mx2) : 1.0f;
           if (need) {
@@ -285,46 +300,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      // P buffer s is free once PV_{j-2} has completed
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(pv_done + s, ((j - 2) >> 1) & 1, abort_flag, g.dev_status))) { ok = false; break; }
-      uint8_t* Pbuf = sP + s * Lay::PB;
-      float rs = 0.f;
+      // P = 2^(s*C - m): packed fp32x2 FMAs; one pair in four on the FMA pipe
+      // (polynomial), the rest on MUFU; four packed partial row sums.
+      const uint64_t NM = f2(-m, -m);
+      uint64_t acc[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
+      uint32_t pk[64];  // the row of P: 128 keys as bf16 pairs
+#pragma unroll
+      for (int w = 0; w < 64; ++w) pk[w] = 0u;
 #pragma unroll
       for (int q = 0; q < TILE / 8; ++q) {
-        uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c0 = q * 8 + 2 * e;
-          float p0 = fast_exp2(fmaf(sv[c0], C, -m));
-          float p1 = fast_exp2(fmaf(sv[c0 + 1], C, -m));
-          if (klen != TILE) {
+          const uint64_t x = f2_fma(f2(sv[c0], sv[c0 + 1]), C2, NM);
+          float p0, p1;
+          if ((POLY_PAIRS >> e) & 1) {
+            f2_split(exp2_poly_f2(x), p0, p1);
+          } else {
+            float x0, x1;
+            f2_split(x, x0, x1);
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          if (!full) {
             p0 = c0 < klen ? p0 : 0.f;
             p1 = c0 + 1 < klen ? p1 : 0.f;
           }
-          rs += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          acc[e] = f2_add(acc[e], f2(p0, p1));
+          if (NSUB == 1 || sub == 0) pk[c0 / 2] = pack_bf16x2_rn(p0, p1);
+          else pk[(TILE + c0) / 2] = pack_bf16x2_rn(p0, p1);
         }
-        const int key_chunk = sub * (TILE / 8) + q;  // 8-key chunk within the 128-key block
-        const int bx = key_chunk >> 3, qq = key_chunk & 7;
-        *reinterpret_cast<uint4*>(Pbuf + bx * (BM * 128) + r * 128 + ((qq ^ (r & 7)) << 4)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      if (NSUB > 1) {  // the other query tile's keys: zero
-#pragma unroll
-        for (int q = 0; q < TILE / 8; ++q) {
-          const int key_chunk = (1 - sub) * (TILE / 8) + q;
-          const int bx = key_chunk >> 3, qq = key_chunk & 7;
-          *reinterpret_cast<uint4*>(Pbuf + bx * (BM * 128) + r * 128 + ((qq ^ (r & 7)) << 4)) =
-              make_uint4(0, 0, 0, 0);
-        }
+      float rs;
+      {
+        const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
+        float lo, hi;
+        f2_split(f2_add(a01, a23), lo, hi);
+        rs = lo + hi;
       }
       l += rs;
-      fence_proxy_async_smem();
+      tmem_st64(lane_addr + s * BN, pk);  // P_j over the first half of S_j
       tc_fence_before();
       mbar_arrive(p_full + s);
     }
     // epilogue: O / l -> bf16
-    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, g.dev_status))) {
+    if (ok && n > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, g.dev_status))) {
       tc_fence_after();
       const float inv = row_valid ? 1.0f / l : 0.f;
       const bool in_range = qb * BM + r < g.n_cap;
@@ -333,14 +356,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
         tmem_ld32(lane_addr + 2 * BN + c * 32, u);
-        uint32_t pk[16];
+        uint32_t o[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(u[2 * e]) * inv, __uint_as_float(u[2 * e + 1]) * inv);
+          o[e] = pack_bf16x2_rn(__uint_as_float(u[2 * e]) * inv, __uint_as_float(u[2 * e + 1]) * inv);
         if (in_range) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
       }
       if (prm.lse && in_range) prm.lse[row0 + r] = row_valid ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
@@ -374,6 +397,10 @@ cudaError_t launch_t(const LayerGeom& g, const void* qp, const void* kp, const v
 
 }  // namespace
 
+cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
+                                    const int32_t* idx, int k_cap, float scale, void* op, float* lse,
+                                    cudaStream_t s);
+
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, int k_cap, float scale, void* op, float* lse, cudaStream_t s) {
   AttnParams prm;
@@ -382,9 +409,8 @@ cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* k
   prm.idx = idx;
   prm.op = reinterpret_cast<__nv_bfloat16*>(op);
   prm.lse = lse;
-  if (g.d == 128 && g.tile == 128) return launch_t<128, 128>(g, qp, kp, vp, prm, s);
-  if (g.d == 128 && g.tile == 64) return launch_t<128, 64>(g, qp, kp, vp, prm, s);
-  if (g.d == 64 && g.tile == 128) return launch_t<64, 128>(g, qp, kp, vp, prm, s);
+  if (g.tile == 128) return launch_sparse_attn_pair(g, qp, kp, vp, idx, k_cap, scale, op, lse, s);
+  if (g.d == 128) return launch_t<128, 64>(g, qp, kp, vp, prm, s);
   return launch_t<64, 64>(g, qp, kp, vp, prm, s);
 }
 

@@ -1,0 +1,475 @@
+// Tile-skipping sparse attention for 128-token tiles, two query tiles per CTA
+// (Veda summary 2.3, Hardware-Efficient Implementation: only the kept
+// key/value tiles are loaded; here each loaded tile also serves both query
+// tiles of the CTA when both kept it).
+//
+// A CTA owns query tiles A = 2c and B = 2c+1 of one head. Their kept-tile
+// lists are merged into one ascending sequence (the union); every union tile
+// is loaded by TMA exactly once, and S = Q K^T / O += P V are issued only for
+// the query tile(s) that kept it. Neighbouring query tiles keep mostly the
+// same key tiles (spatio-temporal locality), so the union is much shorter
+// than the two lists together and each K/V byte from L2 feeds up to twice the
+// tensor work of a one-tile CTA.
+//
+// Roles (384 threads):
+//   warps 0-3 / 4-7  softmax of query tile A / B: thread owns one row (TMEM
+//                    lane). S_A in TMEM columns [0,128), S_B [128,256); P is
+//                    written back as bf16 pairs over the second half of its
+//                    S; O_A at [256, 256+D), O_B after it.
+//   warp 8           K producer (Q_A, Q_B once; then the union's K tiles)
+//   warp 9           MMA issuer (one thread)
+//   warp 10          V producer (the union's V tiles)
+//   warp 11          idle
+// MMA order per union tile e: for A then B: (if the tile kept before e is
+// pending) wait P, issue P V for it; (if the query tile kept e) issue S. So
+// softmax A of tile e runs while the tensor core does B's P V and S, and the
+// V slot of every union tile is released one step later, in order (no ring
+// can fill with tiles whose consumer is far ahead).
+//
+// Every mbarrier wait is bounded (VEDA_WAIT_LIMIT_NS); on expiry the CTA
+// records VEDA_ERR_TIMEOUT, drains what it issued, frees its TMEM and exits.
+#include <climits>
+
+#include "veda_internal.cuh"
+
+namespace veda {
+namespace {
+
+constexpr int BM = 128;               // rows per query tile
+constexpr int BN = 128;               // keys per tile
+constexpr int KST = 2, VST = 3;       // K and V ring stages
+constexpr float RESCALE_LOG2 = 8.0f;  // rescale O only when the max grows by > 2^8
+constexpr int POLY_PAIRS = 0x8;       // which pair of every four runs its exp2 on the FMA pipe
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int NUM_THREADS = 384;
+
+template <int D>
+struct PairLayout {
+  static constexpr int QB = BM * D * 2;
+  static constexpr int KB = BN * D * 2;
+  static constexpr int OFF_Q = 0;  // Q_A, Q_B
+  static constexpr int OFF_K = 2 * QB;
+  static constexpr int OFF_V = OFF_K + KST * KB;
+  static constexpr int OFF_BAR = OFF_V + VST * KB;
+  // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], pv_done[2], drain
+  static constexpr int NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;
+};
+
+struct PairParams {
+  int32_t k_cap;
+  float scale_log2;
+  const int32_t* idx;
+  __nv_bfloat16* op;
+  float* lse;
+};
+
+// j-th kept tile of a list (dense path: j), clamped into [0, nt); an
+// out-of-range entry is reported when `status` is given.
+__device__ __forceinline__ int list_tile(const int32_t* row, int j, int nt, int32_t* status) {
+  if (!row) return j;
+  int t = __ldg(row + j);
+  if (t < 0 || t >= nt) {
+    if (status) report(status, VEDA_ERR_BAD_INDEX);
+    t = 0;
+  }
+  return t;
+}
+
+// Walks the merge of two kept-tile lists: each call yields the next tile and
+// which of the two query tiles kept it. Every entry of both lists is visited
+// exactly once; equal entries are merged.
+struct UnionWalk {
+  const int32_t* la;
+  const int32_t* lb;
+  int ka, kb, ia, ib, nt;
+  int ta, tb;
+  int32_t* status;
+  __device__ UnionWalk(const int32_t* a, int na, const int32_t* b, int nb, int nt_, int32_t* st)
+      : la(a), lb(b), ka(na), kb(nb), ia(0), ib(0), nt(nt_), status(st) {
+    ta = ka > 0 ? list_tile(la, 0, nt, status) : INT_MAX;
+    tb = kb > 0 ? list_tile(lb, 0, nt, nullptr) : INT_MAX;
+  }
+  __device__ bool next(int& t, bool& ma, bool& mb) {
+    if (ia >= ka && ib >= kb) return false;
+    t = ta < tb ? ta : tb;
+    ma = ta == t;
+    mb = tb == t;
+    if (ma) ta = ++ia < ka ? list_tile(la, ia, nt, status) : INT_MAX;
+    if (mb) tb = ++ib < kb ? list_tile(lb, ib, nt, nullptr) : INT_MAX;
+    return true;
+  }
+};
+
+// Maximum of one 64-key half h of a row of S over the valid keys (all of
+// them unless !FULL, then keys below `klen`): eight 3-input max chains.
+template <bool FULL>
+__device__ __forceinline__ float half_max(const uint32_t (&u)[64], int h, int klen) {
+  float pm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 64; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k0 = 64 * h + c + i, k1 = k0 + 8;
+      const float v0 = (FULL || k0 < klen) ? __uint_as_float(u[c + i]) : -INFINITY;
+      const float v1 = (FULL || k1 < klen) ? __uint_as_float(u[c + 8 + i]) : -INFINITY;
+      pm[i] = fmax3(pm[i], v0, v1);
+    }
+  return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+}
+
+// P = 2^(s*C - m) for one 64-key half h of the row as 32 bf16 pairs, with
+// four packed partial row sums. Pairs selected by POLY_PAIRS (per group of
+// four) use the FMA-pipe polynomial, the rest MUFU ex2. Keys at or past
+// `klen` get P = 0 unless FULL.
+template <bool FULL>
+__device__ __forceinline__ void half_p(const uint32_t (&u)[64], int h, int klen, uint64_t C2, uint64_t NM,
+                                       uint64_t (&acc)[4], uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int w = 0; w < 32; ++w) {
+    const int k0 = 64 * h + 2 * w;
+    const uint64_t x = f2_fma(f2(__uint_as_float(u[2 * w]), __uint_as_float(u[2 * w + 1])), C2, NM);
+    float p0, p1;
+    if ((POLY_PAIRS >> (w & 3)) & 1) {
+      f2_split(exp2_poly_f2(x), p0, p1);
+    } else {
+      float x0, x1;
+      f2_split(x, x0, x1);
+      p0 = fast_exp2(x0);
+      p1 = fast_exp2(x1);
+    }
+    if (!FULL) {
+      p0 = k0 < klen ? p0 : 0.f;
+      p1 = k0 + 1 < klen ? p1 : 0.f;
+    }
+    acc[w & 3] = f2_add(acc[w & 3], f2(p0, p1));
+    pk[w] = pack_bf16x2_rn(p0, p1);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    sparse_attn_pair_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ CUtensorMap tmQ,
+                            const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                            const PairParams prm) {
+  using Lay = PairLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+
+  const int cp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * g.heads + h;
+  const HeadGeom& hg = g.h[h];
+  const int nt = hg.nt;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qa = 2 * cp, qbt = 2 * cp + 1;  // the two query tiles
+  const long long rowA = (long long)bh * g.n_cap + (long long)qa * BM;
+
+  if (qa >= nt) {  // both query tiles are padding: zero output rows
+    for (int i = threadIdx.x; i < 2 * BM * D / 8; i += NUM_THREADS) {
+      const int r = i / (D / 8);
+      if (qa * BM + r < g.n_cap)
+        reinterpret_cast<uint4*>(prm.op + (rowA + r) * D)[i % (D / 8)] = make_uint4(0, 0, 0, 0);
+    }
+    if (prm.lse)
+      for (int r = threadIdx.x; r < 2 * BM; r += NUM_THREADS)
+        if (qa * BM + r < g.n_cap) prm.lse[rowA + r] = 0.f;
+    return;
+  }
+  const bool has_b = qbt < nt;
+  const int n = hg.k;
+  const int kA = n, kB = has_b ? n : 0;
+  const int32_t* listA = prm.idx ? prm.idx + ((long long)bh * g.nt_cap + qa) * prm.k_cap : nullptr;
+  const int32_t* listB = prm.idx ? prm.idx + ((long long)bh * g.nt_cap + (has_b ? qbt : qa)) * prm.k_cap : nullptr;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* s_full = v_empty + VST;  // [2]
+  uint64_t* p_full = s_full + 2;     // [2], 128 arrivals each
+  uint64_t* pv_done = p_full + 2;    // [2]
+  uint64_t* mma_drain = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < Lay::NUM_BARS; ++i) {
+      uint64_t* bar = bars + i;
+      mbar_init(bar, (bar == p_full || bar == p_full + 1) ? 128 : 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8 || warp == 10) {
+    // ----------------------------------------------------------- producers
+    if (lane == 0) {
+      const bool is_k = warp == 8;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const int ST = is_k ? KST : VST;
+      uint8_t* ring = smem + (is_k ? Lay::OFF_K : Lay::OFF_V);
+      tma_prefetch_desc(map);
+      if (is_k) {
+        tma_prefetch_desc(&tmQ);
+        mbar_expect_tx(q_full, 2 * Lay::QB);
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tma_load_3d(smem + Lay::OFF_Q + bx * BM * 128, &tmQ, q_full, bx * 64, qa * BM, bh);
+          tma_load_3d(smem + Lay::OFF_Q + Lay::QB + bx * BM * 128, &tmQ, q_full, bx * 64, qbt * BM, bh);
+        }
+      }
+      UnionWalk uw(listA, kA, listB, kB, nt, is_k ? g.dev_status : nullptr);
+      int t, e = 0;
+      bool ma, mb;
+      while (uw.next(t, ma, mb)) {
+        const int st = e % ST;
+        if (e >= ST && !mbar_wait(empty + st, ((e - ST) / ST) & 1, abort_flag, g.dev_status)) break;
+        mbar_expect_tx(full + st, Lay::KB);
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(ring + st * Lay::KB + bx * BN * 128, map, full + st, bx * 64, t * BN, bh);
+        ++e;
+      }
+      if (*abort_flag) {  // let every copy this warp started land before exiting
+        if (is_k) mbar_wait_drain(q_full, 0, VEDA_WAIT_LIMIT_NS);
+        for (int x = e - ST < 0 ? 0 : e - ST; x < e; ++x)
+          mbar_wait_drain(full + x % ST, (x / ST) & 1, VEDA_WAIT_LIMIT_NS);
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(BM, D, false, true);
+      const uint32_t aQ = smem_u32(smem + Lay::OFF_Q);
+      const uint32_t aK = smem_u32(smem + Lay::OFF_K);
+      const uint32_t aV = smem_u32(smem + Lay::OFF_V);
+      bool pend[2] = {false, false};
+      int js[2] = {0, 0};  // S issued per query tile
+      int prev_e = -1;
+      bool ok = mbar_wait(q_full, 0, abort_flag, g.dev_status);
+      if (ok) tc_fence_after();
+      // P V for the tile kept at union position prev_e by query tile r
+      auto issue_pv = [&](int r) -> bool {
+        if (!mbar_wait(p_full + r, (js[r] - 1) & 1, abort_flag, g.dev_status)) return false;
+        if (!mbar_wait(v_full + prev_e % VST, (prev_e / VST) & 1, abort_flag, g.dev_status)) return false;
+        tc_fence_after();
+        const uint32_t o_col = 2 * BN + r * D, s_col = r * BN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ts(tmem + o_col, tmem + s_col + 64 + kk * 8,
+                       sdesc_sw128(aV + (prev_e % VST) * Lay::KB + kk * 2048, BN * 128, 1024), idesc_o,
+                       (js[r] > 1 || kk > 0) ? 1u : 0u);
+        umma_commit(pv_done + r);
+        pend[r] = false;
+        return true;
+      };
+      UnionWalk uw(listA, kA, listB, kB, nt, nullptr);
+      int t, e = 0;
+      bool mem[2];
+      while (ok && uw.next(t, mem[0], mem[1])) {
+        const int st = e % KST;
+        if (!mbar_wait(k_full + st, (e / KST) & 1, abort_flag, g.dev_status)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          if (pend[r] && !(ok = issue_pv(r))) break;
+          if (mem[r]) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+              umma_bf16_ss(tmem + r * BN, sdesc_sw128(aQ + r * Lay::QB + off, 16, 1024),
+                           sdesc_sw128(aK + st * Lay::KB + off, 16, 1024), idesc_s, kk > 0);
+            }
+            umma_commit(s_full + r);
+            js[r]++;
+            pend[r] = true;
+          }
+        }
+        if (!ok) break;
+        if (prev_e >= 0) umma_commit(v_empty + prev_e % VST);  // all P V of prev_e issued
+        umma_commit(k_empty + st);
+        prev_e = e;
+        ++e;
+      }
+      for (int r = 0; r < 2 && ok; ++r)
+        if (pend[r]) ok = issue_pv(r);
+      umma_commit(mma_drain);
+      mbar_wait_drain(mma_drain, 0, VEDA_WAIT_LIMIT_NS);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------- softmax
+    const int r = warp / 4;              // query tile A (0) or B (1)
+    const int row = threadIdx.x % BM;    // row in the tile = TMEM lane
+    const int a = r ? qbt : qa;
+    const int kr = r ? kB : kA;
+    const int32_t* my_list = r ? listB : listA;
+    const bool row_valid = a < nt && row < tile_len(hg, g.T, a);
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+    const uint32_t s_col = r * BN, o_col = 2 * BN + r * D;
+    const float C = prm.scale_log2;
+    const uint64_t C2 = f2(C, C);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    int kt_next = kr > 0 ? list_tile(my_list, 0, nt, nullptr) : 0;
+    for (int j = 0; j < kr; ++j) {
+      const int kt = kt_next;
+      if (j + 1 < kr) kt_next = list_tile(my_list, j + 1, nt, nullptr);  // prefetch the next entry
+      const int klen = tile_len(hg, g.T, kt);
+      const bool full = klen >= BN;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + r, j & 1, abort_flag, g.dev_status))) { ok = false; break; }
+      tc_fence_after();
+      // S row max: keys [0,64) then [64,128); the second half stays in registers
+      uint32_t u1[64];
+      float mx;
+      {
+        uint32_t u0[64];
+        tmem_ld64(lane_addr + s_col, u0);
+        mx = full ? half_max<true>(u0, 0, klen) : half_max<false>(u0, 0, klen);
+      }
+      tmem_ld64(lane_addr + s_col + 64, u1);
+      mx = fmaxf(mx, full ? half_max<true>(u1, 1, klen) : half_max<false>(u1, 1, klen));
+      const float mx2 = mx * C;
+      if (j == 0) {
+        m = mx2;
+      } else {
+        const bool need = mx2 > m + RESCALE_LOG2;
+        if (__any_sync(0xffffffffu, need)) {
+          // O must hold P V of the previous tile before it is rescaled
+          if (!__all_sync(0xffffffffu, mbar_wait(pv_done + r, (j - 1) & 1, abort_flag, g.dev_status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float alpha = need ? fast_exp2(m - mx2) : 1.0f;
+          if (need) {
+            l *= alpha;
+            m = mx2;
+          }
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + o_col + c * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(lane_addr + o_col + c * 32, o);
+          }
+        }
+      }
+      const uint64_t NM = f2(-m, -m);
+      uint64_t acc[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
+      // P (bf16 pairs) goes to columns [64,128) of S: keys [64,128) first
+      // (from registers; their S columns are read already) into [96,128),
+      // then keys [0,64), re-read from columns [0,64), into [64,96).
+      {
+        uint32_t pk[32];
+        if (full) half_p<true>(u1, 1, klen, C2, NM, acc, pk);
+        else half_p<false>(u1, 1, klen, C2, NM, acc, pk);
+        tmem_st32(lane_addr + s_col + 96, pk);
+      }
+      {
+        uint32_t u0[64], pk[32];
+        tmem_ld64(lane_addr + s_col, u0);
+        if (full) half_p<true>(u0, 0, klen, C2, NM, acc, pk);
+        else half_p<false>(u0, 0, klen, C2, NM, acc, pk);
+        tmem_st32(lane_addr + s_col + 64, pk);
+      }
+      {
+        float lo, hi;
+        f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
+        l += lo + hi;
+      }
+      tc_fence_before();
+      mbar_arrive(p_full + r);
+    }
+    // epilogue: O / l -> bf16
+    const long long orow_i = rowA + (long long)r * BM + row;
+    const bool in_range = a * BM + row < g.n_cap;
+    if (kr == 0) {  // query tile beyond this head's tiles: zero rows
+      if (in_range) {
+        uint4* dst = reinterpret_cast<uint4*>(prm.op + orow_i * D);
+#pragma unroll
+        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+        if (prm.lse) prm.lse[orow_i] = 0.f;
+      }
+    } else if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done + r, (kr - 1) & 1, abort_flag, g.dev_status))) {
+      tc_fence_after();
+      const float inv = row_valid ? 1.0f / l : 0.f;
+      __nv_bfloat16* orow = prm.op + orow_i * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(lane_addr + o_col + c * 32, u);
+        uint32_t o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          o[e] = pack_bf16x2_rn(__uint_as_float(u[2 * e]) * inv, __uint_as_float(u[2 * e + 1]) * inv);
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+        }
+      }
+      if (prm.lse && in_range) prm.lse[orow_i] = row_valid ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_pair_t(const LayerGeom& g, const void* qp, const void* kp, const void* vp, const PairParams& prm,
+                          cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t rows = (uint64_t)g.n_cap, planes = (uint64_t)g.B * g.heads;
+  if (encode_tensor_map_3d_bf16(&tq, qp, D, rows, planes, 64, BM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_bf16(&tk, kp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_bf16(&tv, vp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto kern = sparse_attn_pair_kernel<D>;
+  const int smem = PairLayout<D>::SMEM_ALLOC;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((g.nt_cap + 1) / 2, g.heads, g.B);
+  kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, tv, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// 128-token tiles: two query tiles per CTA sharing the loads of their union.
+cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
+                                    const int32_t* idx, int k_cap, float scale, void* op, float* lse,
+                                    cudaStream_t s) {
+  PairParams prm;
+  prm.k_cap = k_cap;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.idx = idx;
+  prm.op = reinterpret_cast<__nv_bfloat16*>(op);
+  prm.lse = lse;
+  if (g.d == 128) return launch_pair_t<128>(g, qp, kp, vp, prm, s);
+  return launch_pair_t<64>(g, qp, kp, vp, prm, s);
+}
+
+}  // namespace veda

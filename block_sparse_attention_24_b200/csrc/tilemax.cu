@@ -178,12 +178,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (it >> 1) & 1, abort_flag, g.dev_status))) break;
       tc_fence_after();
       float sv[BN];
+      {
+        uint32_t u[BN];
+        tmem_ld128(lane_addr + s * BN, u);
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(lane_addr + s * BN + c * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < BN; ++e) sv[e] = __uint_as_float(u[e]);
       }
       tc_fence_before();
       mbar_arrive(s_free + s);  // S buffer may be overwritten now
@@ -193,16 +192,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = 0; u < NSUB; ++u) {
         const int kt = kb * NSUB + u;
         const int klen = kt < nt ? tile_len(hg, g.T, kt) : 0;
-        float mx = -INFINITY;
+        float* x = sv + u * TILE;
+        if (klen < TILE) {  // padded or missing key tile: mask past the valid prefix
 #pragma unroll
-        for (int c = 0; c < TILE; ++c) mx = fmaxf(mx, c < klen ? sv[u * TILE + c] : -INFINITY);
+          for (int c = 0; c < TILE; ++c) x[c] = c < klen ? x[c] : -INFINITY;
+        }
+        float mx;
+        {
+          float pm[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pm[i] = fmaxf(x[i], x[i + 8]);
+#pragma unroll
+          for (int c = 16; c < TILE; c += 16)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], x[c + i], x[c + 8 + i]);
+          mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+        }
         if (!pass2) {
           if (klen > 0) {
             const float mnew = fmaxf(m, mx * C);
-            float acc = 0.f;
+            const uint64_t C2 = f2(C, C), NM = f2(-mnew, -mnew);
+            uint64_t acc[4];
 #pragma unroll
-            for (int c = 0; c < TILE; ++c) acc += c < klen ? fast_exp2(fmaf(sv[u * TILE + c], C, -mnew)) : 0.f;
-            l = l * fast_exp2(m - mnew) + acc;
+            for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < TILE; c += 8) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint64_t y = f2_fma(f2(x[c + 2 * e], x[c + 2 * e + 1]), C2, NM);
+                uint64_t p;
+                if (e & 1) {
+                  p = exp2_poly_f2(y);
+                } else {
+                  float y0, y1;
+                  f2_split(y, y0, y1);
+                  p = f2(fast_exp2(y0), fast_exp2(y1));
+                }
+                if (klen < TILE) {
+                  float p0, p1;
+                  f2_split(p, p0, p1);
+                  p = f2(c + 2 * e < klen ? p0 : 0.f, c + 2 * e + 1 < klen ? p1 : 0.f);
+                }
+                acc[e] = f2_add(acc[e], p);
+              }
+            }
+            float lo, hi;
+            f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
+            l = l * fast_exp2(m - mnew) + (lo + hi);
             m = mnew;
           }
         } else {
