@@ -20,11 +20,12 @@
 //   warp 9           MMA issuer (one thread)
 //   warp 10          V producer (the union's V tiles)
 //   warp 11          idle
-// MMA order per union tile e: for A then B: (if the tile kept before e is
-// pending) wait P, issue P V for it; (if the query tile kept e) issue S. So
-// softmax A of tile e runs while the tensor core does B's P V and S, and the
-// V slot of every union tile is released one step later, in order (no ring
-// can fill with tiles whose consumer is far ahead).
+// MMA order per union tile e: for each query tile that kept e: wait for its
+// P of the previous union tile (if it kept that one), issue its P V, issue S
+// for e; then for a query tile that did not keep e, issue its pending P V.
+// So one query tile's softmax runs while the tensor core works for the
+// other, and the V slot of every union tile is released one step later, in
+// order (no ring can fill with tiles whose consumer is far ahead).
 //
 // Every mbarrier wait is bounded (VEDA_WAIT_LIMIT_NS); on expiry the CTA
 // records VEDA_ERR_TIMEOUT, drains what it issued, frees its TMEM and exits.
@@ -39,9 +40,13 @@ constexpr int BM = 128;               // rows per query tile
 constexpr int BN = 128;               // keys per tile
 constexpr int KST = 2, VST = 3;       // K and V ring stages
 constexpr float RESCALE_LOG2 = 8.0f;  // rescale O only when the max grows by > 2^8
-constexpr int POLY_PAIRS = 0x8;       // which pair of every four runs its exp2 on the FMA pipe
+constexpr int POLY_PAIRS = 0x0;       // which pairs of every four run their exp2 on the FMA pipe
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_THREADS = 384;
+// Registers per thread after the split: softmax warpgroups (2 x 128 threads)
+// and the producer/MMA warpgroup (128 threads); 2*128*216 + 128*72 = 64,512
+// = the 384*168 the launch reserves.
+constexpr int REGS_SOFTMAX = 216, REGS_ROLES = 72;
 
 template <int D>
 struct PairLayout {
@@ -214,7 +219,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+  regs_lower<REGS_ROLES>();
   if (warp == 8 || warp == 10) {
     // ----------------------------------------------------------- producers
     if (lane == 0) {
@@ -287,21 +293,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int st = e % KST;
         if (!mbar_wait(k_full + st, (e / KST) & 1, abort_flag, g.dev_status)) break;
         tc_fence_after();
+        // query tiles that kept tile e: finish their previous P V (P shares
+        // the S columns), then S for tile e
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
+          if (!mem[r]) continue;
           if (pend[r] && !(ok = issue_pv(r))) break;
-          if (mem[r]) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-              umma_bf16_ss(tmem + r * BN, sdesc_sw128(aQ + r * Lay::QB + off, 16, 1024),
-                           sdesc_sw128(aK + st * Lay::KB + off, 16, 1024), idesc_s, kk > 0);
-            }
-            umma_commit(s_full + r);
-            js[r]++;
-            pend[r] = true;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+            umma_bf16_ss(tmem + r * BN, sdesc_sw128(aQ + r * Lay::QB + off, 16, 1024),
+                         sdesc_sw128(aK + st * Lay::KB + off, 16, 1024), idesc_s, kk > 0);
           }
+          umma_commit(s_full + r);
+          js[r]++;
+          pend[r] = true;
         }
+        if (!ok) break;
+        // the other query tile: release its P V of tile e-1 only now, so its
+        // softmax overlaps the S just issued
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+          if (!mem[r] && pend[r] && !(ok = issue_pv(r))) break;
         if (!ok) break;
         if (prev_e >= 0) umma_commit(v_empty + prev_e % VST);  // all P V of prev_e issued
         umma_commit(k_empty + st);
@@ -313,7 +326,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       umma_commit(mma_drain);
       mbar_wait_drain(mma_drain, 0, VEDA_WAIT_LIMIT_NS);
     }
-  } else if (warp < 8) {
+  }
+  } else {
+    regs_raise<REGS_SOFTMAX>();
     // ------------------------------------------------------------- softmax
     const int r = warp / 4;              // query tile A (0) or B (1)
     const int row = threadIdx.x % BM;    // row in the tile = TMEM lane
@@ -327,24 +342,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint64_t C2 = f2(C, C);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    int kt_next = kr > 0 ? list_tile(my_list, 0, nt, nullptr) : 0;
+    // next list entry, loaded one iteration ahead and range-clamped only when
+    // used, so its load latency never stalls the current iteration
+    int raw_next = (kr > 0 && my_list) ? __ldg(my_list) : 0;
     for (int j = 0; j < kr; ++j) {
-      const int kt = kt_next;
-      if (j + 1 < kr) kt_next = list_tile(my_list, j + 1, nt, nullptr);  // prefetch the next entry
+      const int raw = my_list ? raw_next : j;
+      if (my_list && j + 1 < kr) raw_next = __ldg(my_list + j + 1);
+      const int kt = (raw >= 0 && raw < nt) ? raw : 0;
       const int klen = tile_len(hg, g.T, kt);
       const bool full = klen >= BN;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + r, j & 1, abort_flag, g.dev_status))) { ok = false; break; }
       tc_fence_after();
-      // S row max: keys [0,64) then [64,128); the second half stays in registers
-      uint32_t u1[64];
+      // the whole S row in registers: one TMEM load
+      uint32_t u[BN];
+      tmem_ld128(lane_addr + s_col, u);
       float mx;
       {
-        uint32_t u0[64];
-        tmem_ld64(lane_addr + s_col, u0);
-        mx = full ? half_max<true>(u0, 0, klen) : half_max<false>(u0, 0, klen);
+        uint32_t (&u0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[0]);
+        uint32_t (&u1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[64]);
+        mx = full ? fmaxf(half_max<true>(u0, 0, klen), half_max<true>(u1, 1, klen))
+                  : fmaxf(half_max<false>(u0, 0, klen), half_max<false>(u1, 1, klen));
       }
-      tmem_ld64(lane_addr + s_col + 64, u1);
-      mx = fmaxf(mx, full ? half_max<true>(u1, 1, klen) : half_max<false>(u1, 1, klen));
       const float mx2 = mx * C;
       if (j == 0) {
         m = mx2;
@@ -376,21 +394,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint64_t acc[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
-      // P (bf16 pairs) goes to columns [64,128) of S: keys [64,128) first
-      // (from registers; their S columns are read already) into [96,128),
-      // then keys [0,64), re-read from columns [0,64), into [64,96).
+      // P (bf16 pairs) over columns [64,128) of S (all of S is in registers):
+      // keys [0,64) -> [64,96), keys [64,128) -> [96,128); both stores are
+      // asynchronous and waited for once, before P is announced
       {
-        uint32_t pk[32];
-        if (full) half_p<true>(u1, 1, klen, C2, NM, acc, pk);
-        else half_p<false>(u1, 1, klen, C2, NM, acc, pk);
-        tmem_st32(lane_addr + s_col + 96, pk);
-      }
-      {
-        uint32_t u0[64], pk[32];
-        tmem_ld64(lane_addr + s_col, u0);
-        if (full) half_p<true>(u0, 0, klen, C2, NM, acc, pk);
-        else half_p<false>(u0, 0, klen, C2, NM, acc, pk);
-        tmem_st32(lane_addr + s_col + 64, pk);
+        uint32_t (&u0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[0]);
+        uint32_t (&u1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[64]);
+        uint32_t pk0[32], pk1[32];
+        if (full) half_p<true>(u0, 0, klen, C2, NM, acc, pk0);
+        else half_p<false>(u0, 0, klen, C2, NM, acc, pk0);
+        tmem_st32_async(lane_addr + s_col + 64, pk0);
+        if (full) half_p<true>(u1, 1, klen, C2, NM, acc, pk1);
+        else half_p<false>(u1, 1, klen, C2, NM, acc, pk1);
+        tmem_st32_async(lane_addr + s_col + 96, pk1);
+        tmem_wait_st_keep(pk0, pk1);
       }
       {
         float lo, hi;
