@@ -36,4 +36,5 @@ def small_workloads():
         "odd-d128-t64": synth.custom("odd", 1, 3, 128, 3, 8, 8, 64, [(1, 8, 8), (2, 4, 8), (4, 4, 4)], 0.5, 22),
         "batch2-d64-t128": synth.custom("b2", 2, 2, 64, 4, 8, 8, 128, [(2, 8, 8), (4, 4, 8)], 0.5, 23),
         "d64-t64-padded": synth.custom("p64", 1, 2, 64, 7, 4, 8, 64, [(2, 4, 8), (4, 2, 8)], 0.3, 24),
+        "single-tile": synth.custom("one", 1, 2, 128, 1, 8, 16, 128, [(1, 8, 16), (1, 8, 16)], 1.0, 25),
     }

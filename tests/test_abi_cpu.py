@@ -93,3 +93,17 @@ def test_tile_scores_workspace_size():
     w = synth.config(3)
     L = V.Layer(w.B, w.heads, w.d, w.T, w.H, w.W, w.tile, w.tilings)
     assert V.veda_tile_scores_ws_bytes(L, 64) == 2 * 24 * 1200 * 64 * 4
+
+
+def test_empty_and_oversized_layers_rejected():
+    with pytest.raises(V.VedaError) as e:
+        V.Layer(1, 1, 128, 0, 8, 8, 128, [(2, 8, 8)])
+    assert e.value.code == V.VEDA_ERR_INVALID_ARG and "empty" in str(e.value)
+    with pytest.raises(V.VedaError) as e:
+        V.Layer(0, 1, 128, 4, 8, 8, 128, [(2, 8, 8)])
+    assert e.value.code == V.VEDA_ERR_INVALID_ARG
+    with pytest.raises(V.VedaError) as e:      # 8200 tiles of 64 tokens > the 8192-tile limit
+        V.Layer(1, 1, 128, 8200, 8, 8, 64, [(1, 8, 8)])
+    assert e.value.code == V.VEDA_ERR_UNSUPPORTED and "exceeds" in str(e.value)
+    with pytest.raises(V.VedaError):
+        V.Layer(1, 129, 128, 4, 8, 8, 128, [(2, 8, 8)] * 129)
