@@ -178,7 +178,8 @@ int veda_tile_scores(const veda_layer* L, const float* dq, const float* dk, cons
   const void* ptrs[] = {dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scores, emb_ws};
   const char* names[] = {"dq", "dk", "w1q", "b1q", "w2q", "b2q", "w1k", "b1k", "w2k", "b2k", "scores", "emb_ws"};
   for (int i = 0; i < 12; ++i) VEDA_TRY(check_ptr(ptrs[i], names[i]));
-  if (hidden < 1 || hidden > 256) return fail(VEDA_ERR_UNSUPPORTED, "hidden=%d outside [1, 256]", hidden);
+  if (hidden < 4 || hidden > 256 || hidden % 4)
+    return fail(VEDA_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 4 in [4, 256]", hidden);
   if (out_dim < 4 || out_dim > 128 || out_dim % 4)
     return fail(VEDA_ERR_UNSUPPORTED, "out_dim=%d must be a multiple of 4 in [4, 128]", out_dim);
   return after_launch(veda::launch_tile_scores(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim,

@@ -4,10 +4,10 @@
 //   emb = W2^T GELU(W1^T desc + b1) + b2   per tile, per head, for Q and K
 //   scores[i, j] = scale * emb_q[i] . emb_k[j]
 //
-// Two kernels, both fp32 FFMA (no TF32): an MLP kernel that keeps 32 tile
-// descriptors in shared memory and streams each weight once per CTA, and a
-// 64x64-tiled SGEMM for the score matrix. The embeddings live in the
-// caller's scratch buffer between the two.
+// Two kernels, both fp32 FFMA (no TF32): a register-tiled MLP kernel that
+// keeps 32 tile descriptors in shared memory and streams each weight once
+// per CTA, and a 64x64-tiled SGEMM for the score matrix. The embeddings live
+// in the caller's scratch buffer between the two.
 #include "veda_internal.cuh"
 
 namespace veda {
@@ -18,6 +18,12 @@ constexpr int MLP_ROWS = 32;
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
 // grid (ceil(nt_cap/32), heads, B*2): z%2 == 0 -> query side, 1 -> key side.
+// 32 tile descriptors per CTA, kept transposed in shared memory (input-major)
+// so that a thread's 8 rows are two 16-byte loads. Each of the 128 threads
+// owns an 8-row x 4-column register tile of the current layer (32 fp32
+// accumulators, 32 FMAs per 16-byte weight load); layer 1 is applied in
+// chunks of 128 hidden units, GELU'd and transposed into shared memory for
+// layer 2.
 __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerGeom g, const float* __restrict__ dq,
                                                   const float* __restrict__ dk, const float* __restrict__ w1q,
                                                   const float* __restrict__ b1q, const float* __restrict__ w2q,
@@ -25,10 +31,11 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
                                                   const float* __restrict__ b1k, const float* __restrict__ w2k,
                                                   const float* __restrict__ b2k, int hidden, int out_dim,
                                                   float* __restrict__ emb) {
-  extern __shared__ float sm[];
+  extern __shared__ float4 sm4[];
+  float* sm = reinterpret_cast<float*>(sm4);
   const int din = 3 * g.d;
-  float* xs = sm;                          // [MLP_ROWS][din]
-  float* hs = sm + MLP_ROWS * din;         // [MLP_ROWS][hidden]
+  float* xsT = sm;                          // [din][MLP_ROWS]
+  float* hsT = sm + din * MLP_ROWS;         // [hidden][MLP_ROWS]
   const int h = blockIdx.y;
   const int b = blockIdx.z >> 1;
   const int side = blockIdx.z & 1;
@@ -41,40 +48,90 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
   const float* B2 = (side ? b2k : b2q) + (long long)h * out_dim;
   float* out = emb + ((long long)side * g.B * g.heads + (long long)b * g.heads + h) * g.nt_cap * out_dim;
 
-  for (int i = threadIdx.x; i < MLP_ROWS * din; i += blockDim.x) {
-    const int r = i / din, c = i - r * din;
-    xs[i] = (r0 + r < nt) ? desc[(long long)(r0 + r) * din + c] : 0.f;
+  // transpose-load the descriptors: consecutive threads take consecutive rows
+  for (int i = threadIdx.x; i < MLP_ROWS * (din / 4); i += blockDim.x) {
+    const int r = i % MLP_ROWS, c4 = i / MLP_ROWS;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < nt) v = __ldg(reinterpret_cast<const float4*>(desc + (long long)(r0 + r) * din) + c4);
+    xsT[(4 * c4 + 0) * MLP_ROWS + r] = v.x;
+    xsT[(4 * c4 + 1) * MLP_ROWS + r] = v.y;
+    xsT[(4 * c4 + 2) * MLP_ROWS + r] = v.z;
+    xsT[(4 * c4 + 3) * MLP_ROWS + r] = v.w;
   }
   __syncthreads();
-  // layer 1 + GELU: thread owns hidden units j, j+128
-  for (int j = threadIdx.x; j < hidden; j += blockDim.x) {
-    float acc[MLP_ROWS];
-    const float bj = B1[j];
+  const int rg = threadIdx.x / 32;  // rows rg*8 .. rg*8+7 (one warp per row group)
+  const int cg = threadIdx.x % 32;  // columns cg*4 .. cg*4+3 of a 128-column chunk
+
+  // layer 1 + GELU
+  for (int cb = 0; cb < hidden; cb += 128) {
+    const int c = cb + cg * 4;
+    if (c < hidden) {
+      float acc[8][4];
+      const float4 bias = __ldg(reinterpret_cast<const float4*>(B1 + c));
 #pragma unroll
-    for (int r = 0; r < MLP_ROWS; ++r) acc[r] = bj;
-    for (int i = 0; i < din; ++i) {
-      const float w = __ldg(W1 + (long long)i * hidden + j);
+      for (int r = 0; r < 8; ++r) {
+        acc[r][0] = bias.x;
+        acc[r][1] = bias.y;
+        acc[r][2] = bias.z;
+        acc[r][3] = bias.w;
+      }
+#pragma unroll 4
+      for (int i = 0; i < din; ++i) {
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(W1 + (long long)i * hidden + c));
+        const float4 x0 = *reinterpret_cast<const float4*>(xsT + i * MLP_ROWS + rg * 8);
+        const float4 x1 = *reinterpret_cast<const float4*>(xsT + i * MLP_ROWS + rg * 8 + 4);
+        const float xr[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-      for (int r = 0; r < MLP_ROWS; ++r) acc[r] = fmaf(xs[r * din + i], w, acc[r]);
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(xr[r], wr[e], acc[r][e]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float4 v0, v1;
+        v0.x = gelu_erf(acc[0][e]); v0.y = gelu_erf(acc[1][e]); v0.z = gelu_erf(acc[2][e]); v0.w = gelu_erf(acc[3][e]);
+        v1.x = gelu_erf(acc[4][e]); v1.y = gelu_erf(acc[5][e]); v1.z = gelu_erf(acc[6][e]); v1.w = gelu_erf(acc[7][e]);
+        *reinterpret_cast<float4*>(hsT + (c + e) * MLP_ROWS + rg * 8) = v0;
+        *reinterpret_cast<float4*>(hsT + (c + e) * MLP_ROWS + rg * 8 + 4) = v1;
+      }
     }
-#pragma unroll
-    for (int r = 0; r < MLP_ROWS; ++r) hs[r * hidden + j] = gelu_erf(acc[r]);
   }
   __syncthreads();
   // layer 2
-  for (int j = threadIdx.x; j < out_dim; j += blockDim.x) {
-    float acc[MLP_ROWS];
-    const float bj = B2[j];
+  for (int cb = 0; cb < out_dim; cb += 128) {
+    const int c = cb + cg * 4;
+    if (c >= out_dim) continue;
+    float acc[8][4];
+    const float4 bias = __ldg(reinterpret_cast<const float4*>(B2 + c));
 #pragma unroll
-    for (int r = 0; r < MLP_ROWS; ++r) acc[r] = bj;
+    for (int r = 0; r < 8; ++r) {
+      acc[r][0] = bias.x;
+      acc[r][1] = bias.y;
+      acc[r][2] = bias.z;
+      acc[r][3] = bias.w;
+    }
+#pragma unroll 4
     for (int i = 0; i < hidden; ++i) {
-      const float w = __ldg(W2 + (long long)i * out_dim + j);
+      const float4 wv = __ldg(reinterpret_cast<const float4*>(W2 + (long long)i * out_dim + c));
+      const float4 x0 = *reinterpret_cast<const float4*>(hsT + i * MLP_ROWS + rg * 8);
+      const float4 x1 = *reinterpret_cast<const float4*>(hsT + i * MLP_ROWS + rg * 8 + 4);
+      const float xr[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-      for (int r = 0; r < MLP_ROWS; ++r) acc[r] = fmaf(hs[r * hidden + i], w, acc[r]);
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(xr[r], wr[e], acc[r][e]);
     }
 #pragma unroll
-    for (int r = 0; r < MLP_ROWS; ++r)
-      if (r0 + r < g.nt_cap) out[(long long)(r0 + r) * out_dim + j] = (r0 + r < nt) ? acc[r] : 0.f;
+    for (int r = 0; r < 8; ++r) {
+      const int row = r0 + rg * 8 + r;
+      if (row < g.nt_cap) {
+        const bool v = row < nt;
+        *reinterpret_cast<float4*>(out + (long long)row * out_dim + c) =
+            v ? make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
   }
 }
 

@@ -101,7 +101,7 @@ int veda_trippool(const veda_layer* L, const void* xp, float* desc, cudaStream_t
  *   scores[i, j] = scale * q_i . k_j          (i, j < nt_h), fp32 FFMA.
  * GELU is the exact erf form. Weights fp32: w1 [heads, 3d, hidden],
  * b1 [heads, hidden], w2 [heads, hidden, out_dim], b2 [heads, out_dim];
- * hidden <= 256, out_dim <= 128 and a multiple of 4. emb_ws is caller scratch
+ * hidden <= 256 and out_dim <= 128, both multiples of 4. emb_ws is caller scratch
  * of veda_tile_scores_ws_bytes() bytes (the q and k embeddings). */
 int veda_tile_scores(const veda_layer* L, const float* dq, const float* dk,
                      const float* w1q, const float* b1q, const float* w2q, const float* b2q,
