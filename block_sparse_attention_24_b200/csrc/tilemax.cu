@@ -2,39 +2,41 @@
 // Optimization; 2.3, Training Efficiency: the heat map is built in two
 // passes, on a subset of query tiles).
 //
-// One CTA owns 128 query rows (one 128-token query tile, or two 64-token
-// query tiles) of one selected head and sweeps every key block of the head
-// twice with tcgen05 S = Q K^T:
-//   pass 1: per row, lse = log2-domain log-sum-exp over all valid keys;
+// Two 128-row blocks of selected query tiles share one CTA and every K block
+// load; each sweeps all key blocks twice with tcgen05 S = Q K^T:
+//   pass 1: per row, log2-domain log-sum-exp over all valid keys;
 //   pass 2: per row and key tile, the largest logit minus lse, then the
 //           maximum over the tile's valid rows (warp shuffle, then a shared
 //           order-preserving atomicMax) -> M[a, b] = exp2(.) = max-pooled
 //           softmax probability over the tile region.
-// Roles as in the attention kernel: 4 softmax warps (row r = TMEM lane r), a
-// TMA producer warp with a 3-stage K ring, one MMA-issuing thread, S double
-// buffered in TMEM. A second kernel turns map rows and score rows into KL
-// values, a third averages them in a fixed order.
+// A second kernel turns map rows and score rows into KL values, a third
+// averages them in a fixed order.
 #include "veda_internal.cuh"
 
 namespace veda {
 namespace {
 
 constexpr int BM = 128, BN = 128;
-constexpr int KST = 3;  // K ring stages
-constexpr uint32_t TMEM_COLS = 256;
-constexpr int NUM_THREADS = 192;
+constexpr int KST = 3;                 // K ring stages
+constexpr uint32_t TMEM_COLS = 512;    // S buffers: row-block r, buffer b at (2r + b) * 128
+constexpr int NUM_THREADS = 384;
+// softmax warpgroups 216 registers, producer/MMA warpgroup 72:
+// 2*128*216 + 128*72 = 64,512 = the 384*168 the launch reserves
+constexpr int REGS_SOFTMAX = 216, REGS_ROLES = 72;
+constexpr int POLY_PAIRS = 0xA;        // pass 1: pairs 1 and 3 of every four use the FMA-pipe exp2
 
 template <int D>
 struct MapLayout {
-  static constexpr int QB = BM * D * 2;
+  static constexpr int QB = BM * D * 2;  // one 128-row block of Q
   static constexpr int KB = BN * D * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = QB;
+  static constexpr int OFF_Q = 0;        // row blocks A, B
+  static constexpr int OFF_K = 2 * QB;
   static constexpr int OFF_BAR = OFF_K + KST * KB;
-  static constexpr int NUM_BARS = 1 + 2 * KST + 2 + 2 + 1;  // q_full, k_full/empty, s_full, s_free, drain
+  // q_full, k_full[KST], k_empty[KST], s_full[4], s_free[4], drain
+  static constexpr int NUM_BARS = 1 + 2 * KST + 4 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_PART = (OFF_MISC + 16 + 15) / 16 * 16;
-  static int bytes(int nt_cap) { return OFF_PART + (BM / 64) * nt_cap * 4 + 1024; }
+  static int bytes(int nt_cap, int nsub) { return OFF_PART + 2 * nsub * nt_cap * 4 + 1024; }
 };
 
 struct MapParams {
@@ -54,12 +56,72 @@ __device__ __forceinline__ float unord_f32(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+// Maximum of columns [c0, c0+TILE) of a row of S over the first `klen` of
+// them (all when FULL).
+template <int TILE, bool FULL>
+__device__ __forceinline__ float tile_max(const uint32_t (&u)[BN], int c0, int klen) {
+  float pm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < TILE; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k0 = c + i, k1 = k0 + 8;
+      const float v0 = (FULL || k0 < klen) ? __uint_as_float(u[c0 + k0]) : -INFINITY;
+      const float v1 = (FULL || k1 < klen) ? __uint_as_float(u[c0 + k1]) : -INFINITY;
+      pm[i] = fmax3(pm[i], v0, v1);
+    }
+  return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+}
+
+// Sum over columns [c0, c0+TILE) (the first `klen`, all when FULL) of
+// 2^(s*C - mnew); packed fp32x2 math, part of the exponentials on the FMA pipe.
+template <int TILE, bool FULL>
+__device__ __forceinline__ float tile_expsum(const uint32_t (&u)[BN], int c0, int klen, uint64_t C2, uint64_t NM) {
+  uint64_t acc[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
+#pragma unroll
+  for (int w = 0; w < TILE / 2; ++w) {
+    const int k0 = 2 * w;
+    const uint64_t y = f2_fma(f2(__uint_as_float(u[c0 + k0]), __uint_as_float(u[c0 + k0 + 1])), C2, NM);
+    uint64_t p;
+    if ((POLY_PAIRS >> (w & 3)) & 1) {
+      p = exp2_poly_f2(y);
+    } else {
+      float y0, y1;
+      f2_split(y, y0, y1);
+      p = f2(fast_exp2(y0), fast_exp2(y1));
+    }
+    if (!FULL) {
+      float p0, p1;
+      f2_split(p, p0, p1);
+      p = f2(k0 < klen ? p0 : 0.f, k0 + 1 < klen ? p1 : 0.f);
+    }
+    acc[w & 3] = f2_add(acc[w & 3], p);
+  }
+  float lo, hi;
+  f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
+  return lo + hi;
+}
+
+// One CTA owns two 128-row blocks (A, B) of selected query rows of one head:
+// one 128-token query tile each, or two 64-token query tiles each. Both
+// sweep every key block twice (pass 1: log-sum-exp; pass 2: per key tile
+// max of logit - lse, then max over the tile's rows); each K block is loaded
+// once for both. S of each row block is double-buffered in TMEM, so the MMA
+// for the next key block overlaps the softmax of the current one.
+//   warps 0-3 / 4-7  row block A / B (thread = row = TMEM lane)
+//   warp 8           TMA producer (Q once, then K blocks, 3-stage ring)
+//   warp 9           MMA issuer (one thread)
+//   warps 10-11      idle
 template <int D, int TILE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tilemax_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ MapParams prm) {
   using Lay = MapLayout<D>;
-  constexpr int NSUB = BM / TILE;
+  constexpr int NSUB = BM / TILE;  // query tiles per row block
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -73,40 +135,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n_kb = (nt * TILE + BN - 1) / BN;
   const int iters = 2 * n_kb;
 
-  // query tiles of this CTA
-  int qt[NSUB];
-  bool qv[NSUB];
+  // selected query tiles: entry (2*blockIdx.x + r)*NSUB + s of the row list
+  int qt[2][NSUB];
+  bool qv[2][NSUB];
+  bool rb_valid[2];
 #pragma unroll
-  for (int s = 0; s < NSUB; ++s) {
-    const int r = blockIdx.x * NSUB + s;
-    qv[s] = r < prm.n_rows;
-    int a = qv[s] ? (prm.rows ? __ldg(prm.rows + (long long)hs * prm.n_rows + r) : r) : 0;
-    if (a < 0 || a >= nt) {
-      if (qv[s]) report(g.dev_status, VEDA_ERR_BAD_INDEX);
-      a = 0;
-      qv[s] = false;
+  for (int r = 0; r < 2; ++r) {
+    rb_valid[r] = false;
+#pragma unroll
+    for (int s = 0; s < NSUB; ++s) {
+      const int e = (2 * blockIdx.x + r) * NSUB + s;
+      qv[r][s] = e < prm.n_rows;
+      int a = qv[r][s] ? (prm.rows ? __ldg(prm.rows + (long long)hs * prm.n_rows + e) : e) : 0;
+      if (a < 0 || a >= nt) {
+        if (qv[r][s]) report(g.dev_status, VEDA_ERR_BAD_INDEX);
+        a = 0;
+        qv[r][s] = false;
+      }
+      qt[r][s] = a;
+      rb_valid[r] = rb_valid[r] || qv[r][s];
     }
-    qt[s] = a;
   }
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 1 + KST;
-  uint64_t* s_full = bars + 1 + 2 * KST;
-  uint64_t* s_free = bars + 3 + 2 * KST;
-  uint64_t* drain = bars + 5 + 2 * KST;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* s_full = k_empty + KST;  // [row block * 2 + buffer]
+  uint64_t* s_free = s_full + 4;     // [row block * 2 + buffer], 128 arrivals each
+  uint64_t* drain = s_free + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
-  uint32_t* part = reinterpret_cast<uint32_t*>(smem + Lay::OFF_PART);  // [NSUB][nt_cap] ordered maxima
+  uint32_t* part = reinterpret_cast<uint32_t*>(smem + Lay::OFF_PART);  // [2][NSUB][nt_cap] ordered maxima
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < Lay::NUM_BARS; ++i) mbar_init(bars + i, (i == 3 + 2 * KST || i == 4 + 2 * KST) ? 128 : 1);
+    for (int i = 0; i < Lay::NUM_BARS; ++i) {
+      uint64_t* bar = bars + i;
+      mbar_init(bar, (bar >= s_free && bar < s_free + 4) ? 128 : 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < NSUB * g.nt_cap; i += NUM_THREADS) part[i] = 0u;  // 0 = no contribution
-  if (warp == 5) {
+  for (int i = threadIdx.x; i < 2 * NSUB * g.nt_cap; i += NUM_THREADS) part[i] = 0u;  // 0 = no contribution
+  if (warp == 9) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
@@ -114,16 +185,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
-    if (lane == 0) {
+  if (warp >= 8) {
+    regs_lower<REGS_ROLES>();
+    if (warp == 8 && lane == 0) {
+      // ------------------------------------------------------- producer
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      mbar_expect_tx(q_full, Lay::QB);
+      mbar_expect_tx(q_full, 2 * Lay::QB);
 #pragma unroll
-      for (int s = 0; s < NSUB; ++s)
+      for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_3d(smem + Lay::OFF_Q + bx * BM * 128 + s * TILE * 128, &tmQ, q_full, bx * 64, qt[s] * TILE, bh);
+        for (int s = 0; s < NSUB; ++s)
+#pragma unroll
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_3d(smem + Lay::OFF_Q + r * Lay::QB + bx * BM * 128 + s * TILE * 128, &tmQ, q_full, bx * 64,
+                        qt[r][s] * TILE, bh);
       int issued = 0;
       for (int it = 0; it < iters; ++it) {
         const int st = it % KST;
@@ -140,140 +216,109 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int it = issued - KST < 0 ? 0 : issued - KST; it < issued; ++it)
           mbar_wait_drain(k_full + it % KST, (it / KST) & 1, VEDA_WAIT_LIMIT_NS);
       }
-    }
-  } else if (warp == 5) {
-    if (lane == 0) {
+    } else if (warp == 9 && lane == 0) {
+      // ------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
       const uint32_t aQ = smem_u32(smem + Lay::OFF_Q);
       const uint32_t aK = smem_u32(smem + Lay::OFF_K);
       if (mbar_wait(q_full, 0, abort_flag, g.dev_status)) {
         tc_fence_after();
-        for (int it = 0; it < iters; ++it) {
-          const int s = it & 1, st = it % KST;
-          if (it >= 2 && !mbar_wait(s_free + s, ((it - 2) >> 1) & 1, abort_flag, g.dev_status)) break;
+        bool ok = true;
+        for (int it = 0; it < iters && ok; ++it) {
+          const int st = it % KST, buf = it & 1;
           if (!mbar_wait(k_full + st, (it / KST) & 1, abort_flag, g.dev_status)) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-            umma_bf16_ss(tmem + s * BN, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + st * Lay::KB + off, 16, 1024),
-                         idesc, kk > 0);
+          for (int r = 0; r < 2; ++r) {
+            if (!rb_valid[r]) continue;
+            const int sb = 2 * r + buf;
+            if (it >= 2 && !(ok = mbar_wait(s_free + sb, ((it - 2) >> 1) & 1, abort_flag, g.dev_status))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+              umma_bf16_ss(tmem + sb * BN, sdesc_sw128(aQ + r * Lay::QB + off, 16, 1024),
+                           sdesc_sw128(aK + st * Lay::KB + off, 16, 1024), idesc, kk > 0);
+            }
+            umma_commit(s_full + sb);
           }
-          umma_commit(s_full + s);
-          umma_commit(k_empty + st);
+          if (ok) umma_commit(k_empty + st);
         }
       }
       umma_commit(drain);
       mbar_wait_drain(drain, 0, VEDA_WAIT_LIMIT_NS);
     }
   } else {
-    const int r = threadIdx.x;
-    const int qs = r / TILE;  // query sub-tile of this row
-    const bool row_valid = qv[qs] && (r % TILE) < tile_len(hg, g.T, qt[qs]);
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    regs_raise<REGS_SOFTMAX>();
+    // ------------------------------------------------------------ softmax
+    const int r = warp / 4;                 // row block
+    const int row = threadIdx.x % BM;       // TMEM lane
+    const int qs = row / TILE;              // query tile within the row block
+    const bool row_valid = qv[r][qs] && (row % TILE) < tile_len(hg, g.T, qt[r][qs]);
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float C = prm.scale_log2;
+    const uint64_t C2 = f2(C, C);
     float m = -INFINITY, l = 0.f, lse2 = 0.f;
-    for (int it = 0; it < iters; ++it) {
-      const int s = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (it >> 1) & 1, abort_flag, g.dev_status))) break;
+    for (int it = 0; it < (rb_valid[r] ? iters : 0); ++it) {
+      const int sb = 2 * r + (it & 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, (it >> 1) & 1, abort_flag, g.dev_status))) break;
       tc_fence_after();
-      float sv[BN];
-      {
-        uint32_t u[BN];
-        tmem_ld128(lane_addr + s * BN, u);
-#pragma unroll
-        for (int e = 0; e < BN; ++e) sv[e] = __uint_as_float(u[e]);
-      }
+      uint32_t u[BN];
+      tmem_ld128(lane_addr + sb * BN, u);
       tc_fence_before();
-      mbar_arrive(s_free + s);  // S buffer may be overwritten now
+      mbar_arrive(s_free + sb);  // S buffer may be overwritten now
       const int kb = it % n_kb;
       const bool pass2 = it >= n_kb;
 #pragma unroll
-      for (int u = 0; u < NSUB; ++u) {
-        const int kt = kb * NSUB + u;
+      for (int uu = 0; uu < NSUB; ++uu) {
+        const int kt = kb * NSUB + uu;
         const int klen = kt < nt ? tile_len(hg, g.T, kt) : 0;
-        float* x = sv + u * TILE;
-        if (klen < TILE) {  // padded or missing key tile: mask past the valid prefix
-#pragma unroll
-          for (int c = 0; c < TILE; ++c) x[c] = c < klen ? x[c] : -INFINITY;
-        }
-        float mx;
-        {
-          float pm[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pm[i] = fmaxf(x[i], x[i + 8]);
-#pragma unroll
-          for (int c = 16; c < TILE; c += 16)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], x[c + i], x[c + 8 + i]);
-          mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-        }
+        const bool full = klen >= TILE;
+        const float mx = full ? tile_max<TILE, true>(u, uu * TILE, klen) : tile_max<TILE, false>(u, uu * TILE, klen);
         if (!pass2) {
           if (klen > 0) {
             const float mnew = fmaxf(m, mx * C);
-            const uint64_t C2 = f2(C, C), NM = f2(-mnew, -mnew);
-            uint64_t acc[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < TILE; c += 8) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const uint64_t y = f2_fma(f2(x[c + 2 * e], x[c + 2 * e + 1]), C2, NM);
-                uint64_t p;
-                if (e & 1) {
-                  p = exp2_poly_f2(y);
-                } else {
-                  float y0, y1;
-                  f2_split(y, y0, y1);
-                  p = f2(fast_exp2(y0), fast_exp2(y1));
-                }
-                if (klen < TILE) {
-                  float p0, p1;
-                  f2_split(p, p0, p1);
-                  p = f2(c + 2 * e < klen ? p0 : 0.f, c + 2 * e + 1 < klen ? p1 : 0.f);
-                }
-                acc[e] = f2_add(acc[e], p);
-              }
-            }
-            float lo, hi;
-            f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
-            l = l * fast_exp2(m - mnew) + (lo + hi);
+            const uint64_t NM = f2(-mnew, -mnew);
+            const float sum = full ? tile_expsum<TILE, true>(u, uu * TILE, klen, C2, NM)
+                                   : tile_expsum<TILE, false>(u, uu * TILE, klen, C2, NM);
+            l = l * fast_exp2(m - mnew) + sum;
             m = mnew;
           }
         } else {
           float v = (row_valid && klen > 0) ? fmaf(mx, C, -lse2) : -INFINITY;
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-          if (lane == 0 && kt < nt && v > -INFINITY) atomicMax(part + qs * g.nt_cap + kt, ord_f32(v));
+          if (lane == 0 && kt < nt && v > -INFINITY) atomicMax(part + (r * NSUB + qs) * g.nt_cap + kt, ord_f32(v));
         }
       }
       if (it == n_kb - 1) {
         lse2 = m + __log2f(l);
-        const int rr = blockIdx.x * NSUB + qs;
-        if (prm.lse && rr < prm.n_rows)
-          prm.lse[((long long)hs * prm.n_rows + rr) * TILE + (r % TILE)] = row_valid ? lse2 * 0.69314718055994531f : 0.f;
+        const int e = (2 * blockIdx.x + r) * NSUB + qs;
+        if (prm.lse && e < prm.n_rows)
+          prm.lse[((long long)hs * prm.n_rows + e) * TILE + (row % TILE)] = row_valid ? lse2 * 0.69314718055994531f : 0.f;
       }
     }
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
-  // write the map rows and lse
+  // write the map rows
   if (!*abort_flag) {
 #pragma unroll
-    for (int s = 0; s < NSUB; ++s) {
-      const int rr = blockIdx.x * NSUB + s;
-      if (rr >= prm.n_rows) continue;
-      float* out = prm.tilemap + ((long long)hs * prm.n_rows + rr) * g.nt_cap;
-      for (int b = threadIdx.x; b < g.nt_cap; b += NUM_THREADS) {
-        const uint32_t k = part[s * g.nt_cap + b];
-        out[b] = (b < nt && k != 0u && qv[s]) ? fast_exp2(unord_f32(k)) : 0.f;
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int s = 0; s < NSUB; ++s) {
+        const int e = (2 * blockIdx.x + r) * NSUB + s;
+        if (e >= prm.n_rows) continue;
+        float* out = prm.tilemap + ((long long)hs * prm.n_rows + e) * g.nt_cap;
+        for (int b = threadIdx.x; b < g.nt_cap; b += NUM_THREADS) {
+          const uint32_t k = part[(r * NSUB + s) * g.nt_cap + b];
+          out[b] = (b < nt && k != 0u && qv[r][s]) ? fast_exp2(unord_f32(k)) : 0.f;
+        }
       }
-    }
   }
 }
 
@@ -347,11 +392,12 @@ cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, con
   if (encode_tensor_map_3d_bf16(&tq, qp, D, rows, planes, 64, TILE) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (encode_tensor_map_3d_bf16(&tk, kp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   auto kern = tilemax_kernel<D, TILE>;
-  const int smem = MapLayout<D>::bytes(g.nt_cap);
+  constexpr int NSUB = BM / TILE;
+  const int smem = MapLayout<D>::bytes(g.nt_cap, NSUB);
   if (smem > 232448) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((prm.n_rows + BM / TILE - 1) / (BM / TILE), n_heads_sel, 1);
+  const dim3 grid((prm.n_rows + 2 * NSUB - 1) / (2 * NSUB), n_heads_sel, 1);
   kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, prm);
   return cudaGetLastError();
 }
