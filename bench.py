@@ -200,7 +200,7 @@ def run_ours(args, world, rank, local):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize(device)
-    if True:
+    if True:  # timed region
         host_t0 = datetime.datetime.now()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
@@ -255,6 +255,7 @@ def run_ours(args, world, rank, local):
     step_ms = elapsed / args.steps * 1e3
     value = world * eff_flops / (elapsed / args.steps) / 1e12
     traffic = load_traffic()
+    hbm_stages = frontend_bandwidth(L, layer, stage_ms, unperm_ms, hbm)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, layer, L, budget_s=args.cpu_seconds)
@@ -276,8 +277,10 @@ def run_ours(args, world, rank, local):
                      "unpermute": round(unperm_ms, 3), "tilemap_kl": round(map_ms, 3)},
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": sustained, "unit": UNIT,
                      "frac": round(attn_tflops / sustained, 4), "traffic": traffic,
-                     "kernel": "sparse_attn_kernel<128,128>",
+                     "kernel": "sparse_attn_pair_kernel<128>",
+                     "kernel_source_sha256_16": kernel_source_hash(),
                      "peak_kind": f"bf16 dense sustained ({src}); burst {burst}"},
+        "hbm_stages": hbm_stages,
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
@@ -344,14 +347,50 @@ def run_e2e(V, L, layer, q, k, v, device, eff_flops, args):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
 
+def kernel_source_hash() -> str:
+    import hashlib
+    hsh = hashlib.sha256()
+    for f in ("attn_pair.cu", "veda_internal.cuh"):
+        hsh.update(open(os.path.join(ROOT, "block_sparse_attention_24_b200", "csrc", f), "rb").read())
+    return hsh.hexdigest()[:16]
+
+
 def load_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it
-    matches the current kernel (written by hand from an ncu capture)."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes (read + write) per attention launch at this workload, from
+    the committed ncu summary; None once the kernel source differs from the
+    one the counters were taken on."""
+    p = os.path.join(ROOT, "profiles", "sparse_attn_traffic_153600tok.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d.get("sparse_attn_bytes_per_launch")
+        if d.get("kernel_source_sha256_16") == kernel_source_hash():
+            return d.get("dram_bytes_per_launch")
     return None
+
+
+def frontend_bandwidth(L, layer, stage_ms, unperm_ms, hbm_gbs):
+    """Algorithmic HBM bytes of the bandwidth-bound stages and the achieved
+    rate against the measured HBM copy bandwidth."""
+    Hh, d, B = L.heads, L.d, L.B
+    valid = sum(L.N for _ in range(Hh)) * B          # valid token rows over heads
+    row = d * 2
+    nt_sum = sum(L.nt) * B
+    byts = {
+        # read every original row, write every permuted row (incl. padding), x3 tensors
+        "permute_qkv": 3 * (valid * row + B * Hh * L.n_cap * row),
+        # read the valid rows of Qp and Kp, write [avg|max|min] fp32 per tile
+        "trippool_qk": 2 * (valid * row + nt_sum * 3 * d * 4),
+        # read the scores, write index lists and the dense mask
+        "topk": B * Hh * L.nt_cap * L.nt_cap * 4 + B * Hh * L.nt_cap * (layer.k_cap * 4 + L.nt_cap),
+    }
+    out = {}
+    for k, b in byts.items():
+        ms = stage_ms[k]
+        out[k] = {"bytes": b, "ms": ms, "gbs": round(b / (ms / 1e3) / 1e9, 1),
+                  "frac_of_measured_hbm": round(b / (ms / 1e3) / 1e9 / hbm_gbs, 3)}
+    b = valid * row + B * Hh * L.n_cap * row
+    out["unpermute"] = {"bytes": b, "ms": unperm_ms, "gbs": round(b / (unperm_ms / 1e3) / 1e9, 1),
+                        "frac_of_measured_hbm": round(b / (unperm_ms / 1e3) / 1e9 / hbm_gbs, 3)}
+    return out
 
 
 # ------------------------------------------------------------ CPU oracle
