@@ -72,6 +72,7 @@ int build_geom(const veda_layer* L, veda::LayerGeom* g) {
     if (nt > VEDA_MAX_NT) return fail(VEDA_ERR_UNSUPPORTED, "head %d: %lld tiles exceeds %d", h, nt, VEDA_MAX_NT);
     hg.nt = (int)nt;
     hg.k = 0;
+    hg.padded = (L->T % t.pt) != 0;
     if (nt > nt_cap) nt_cap = (int)nt;
     if (nt * L->tile > n_cap) n_cap = (int)(nt * L->tile);
   }

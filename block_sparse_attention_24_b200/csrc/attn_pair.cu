@@ -342,14 +342,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint64_t C2 = f2(C, C);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // next list entry, loaded one iteration ahead and range-clamped only when
-    // used, so its load latency never stalls the current iteration
-    int raw_next = (kr > 0 && my_list) ? __ldg(my_list) : 0;
+    // A head whose tiles are all full never needs the kept tile's index here.
+    // Otherwise the next list entry is loaded one iteration ahead and
+    // range-clamped only when used, so its latency never stalls an iteration.
+    const bool padded = hg.padded != 0;
+    const int32_t* pad_list = padded ? my_list : nullptr;
+    int raw_next = (kr > 0 && pad_list) ? __ldg(pad_list) : 0;
     for (int j = 0; j < kr; ++j) {
-      const int raw = my_list ? raw_next : j;
-      if (my_list && j + 1 < kr) raw_next = __ldg(my_list + j + 1);
-      const int kt = (raw >= 0 && raw < nt) ? raw : 0;
-      const int klen = tile_len(hg, g.T, kt);
+      int klen = BN;
+      if (padded) {
+        const int raw = pad_list ? raw_next : j;
+        if (pad_list && j + 1 < kr) raw_next = __ldg(pad_list + j + 1);
+        const int kt = (raw >= 0 && raw < nt) ? raw : 0;
+        klen = tile_len(hg, g.T, kt);
+      }
       const bool full = klen >= BN;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + r, j & 1, abort_flag, g.dev_status))) { ok = false; break; }
       tc_fence_after();

@@ -24,6 +24,7 @@ struct HeadGeom {
   int32_t tps;     // tiles per time slab = (H/ph)*(W/pw)
   int32_t nwt;     // tiles along W = W/pw
   int32_t k;       // kept key tiles per query tile (attention / top-k)
+  int32_t padded;  // 1 if p_t does not divide T (the last time slab of tiles is partial)
 };
 
 struct LayerGeom {
