@@ -200,7 +200,7 @@ def run_ours(args, world, rank, local):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize(device)
-    if True:  # timed region
+    if True:  # the timed region
         host_t0 = datetime.datetime.now()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
@@ -486,6 +486,57 @@ def run_reference(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Head-group sweep (8 heads, d=128, 128-token tiles): sparse attention at
+    each keep fraction against the same kernel's dense path, per token count.
+    Prints one JSON object per point (not the benchmark contract line)."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    burst, sustained, _, src = measured_peaks()
+    out = []
+    for tokens in synth.SWEEP_TOKENS:
+        dense_ms = None
+        for keep in sorted(synth.SWEEP_KEEP, reverse=True):
+            w = synth.sweep(tokens, keep)
+            V, L, layer, (q, k, v) = build_layer(w, device)
+            layer.front(q, k, v)
+            torch.cuda.synchronize()
+            kept, allp = kept_pairs(L, layer)
+            flops = 4.0 * L.d * kept
+            args_attn = (L, layer.qp, layer.kp, layer.vp, layer.idx, layer.k, layer.k_cap, layer.attn_scale, layer.op)
+            for _ in range(2):
+                V.veda_sparse_attn(*args_attn)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            e0.record()
+            for _ in range(reps):
+                V.veda_sparse_attn(*args_attn)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            if dense_ms is None:
+                dout = torch.empty_like(layer.op)
+                layer.dense(dout)
+                e0.record()
+                for _ in range(3):
+                    layer.dense(dout)
+                e1.record()
+                torch.cuda.synchronize()
+                dense_ms = e0.elapsed_time(e1) / 3
+                dense_flops = 4.0 * L.d * allp
+                del dout
+            V.veda_check_status(L)
+            rec = {"tokens": w.N, "keep": keep, "sparsity": round(1 - kept / allp, 4), "k": layer.k[0],
+                   "attn_ms": round(ms, 3), "eff_tflops": round(flops / ms / 1e9, 1),
+                   "frac_of_burst_peak": round(flops / ms / 1e9 / burst, 4), "dense_ms": round(dense_ms, 3),
+                   "dense_tflops": round(dense_flops / dense_ms / 1e9, 1), "speedup_vs_dense": round(dense_ms / ms, 2)}
+            print(json.dumps(rec), flush=True)
+            out.append(rec)
+            del layer, q, k, v
+            torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -499,10 +550,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="head-group token/sparsity sweep instead of the step")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps are required")
     world, rank, local = dist_env()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank, local)
     else:

@@ -28,7 +28,7 @@ VEDA_ERR_BAD_INDEX = -5
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
             "veda_topk_mask", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
-            "veda_last_error")
+            "veda_selftest_wait_timeout", "veda_last_error")
 
 
 class VedaError(RuntimeError):
@@ -71,6 +71,7 @@ _lib.veda_topk_mask.argtypes = [_LP, _P, _P, _I, _P, _P, _P]
 _lib.veda_sparse_attn.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
 _lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P, _P, _P, _P, _P]
 _lib.veda_check_status.argtypes = [_LP, _P]
+_lib.veda_selftest_wait_timeout.argtypes = [_LP, ctypes.c_uint32, _P]
 _lib.veda_last_error.restype = ctypes.c_char_p
 for _name in EXPORTED:
     getattr(_lib, _name)
@@ -196,6 +197,10 @@ def veda_full_attn_tilemax(layer: Layer, qp, kp, heads_sel: Sequence[int], qtile
 
 def veda_check_status(layer: Layer, stream=None):
     _check(_lib.veda_check_status(layer.ref, _stream(stream)))
+
+
+def veda_selftest_wait_timeout(layer: Layer, limit_ms: int, stream=None):
+    _check(_lib.veda_selftest_wait_timeout(layer.ref, int(limit_ms), _stream(stream)))
 
 
 def library_path() -> str:

@@ -108,10 +108,11 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t pari
 
 // Waits for the phase of `bar` with parity `parity` to complete. Gives up
 // (returns false) when another warp of the CTA has already given up
-// (*abort != 0) or after VEDA_WAIT_LIMIT_NS, in which case it records
-// VEDA_ERR_TIMEOUT and raises *abort for the rest of the CTA.
+// (*abort != 0), when another CTA has recorded a timeout, or after
+// `limit_ns`, in which case it records VEDA_ERR_TIMEOUT and raises *abort
+// for the rest of the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* status) {
+                                          int32_t* status, uint64_t limit_ns = VEDA_WAIT_LIMIT_NS) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -124,7 +125,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         *abort = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > VEDA_WAIT_LIMIT_NS) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         report(status, VEDA_ERR_TIMEOUT);
         return false;

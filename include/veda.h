@@ -169,6 +169,14 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp,
                            float* tilemap, float* lse, const float* scores,
                            float* kl_rows, float* kl_out, cudaStream_t stream);
 
+/* Diagnostic (no counterpart on the pages): launches one thread that waits,
+ * through the bounded wait every pipeline kernel uses, on a barrier nothing
+ * arrives on. After limit_ms (1..10000) the wait gives up and records
+ * VEDA_ERR_TIMEOUT in L->dev_status; the kernel then returns normally, so a
+ * following veda_check_status reports the timeout and the context remains
+ * usable. Lets callers verify the failure path without faulting a GPU. */
+int veda_selftest_wait_timeout(const veda_layer* L, uint32_t limit_ms, cudaStream_t stream);
+
 /* Synchronises `stream`, returns the first device-side status recorded in
  * L->dev_status (VEDA_OK if none) and clears it. */
 int veda_check_status(const veda_layer* L, cudaStream_t stream);
