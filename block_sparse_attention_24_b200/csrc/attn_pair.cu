@@ -20,9 +20,9 @@
 //   warp 9           MMA issuer (one thread)
 //   warp 10          V producer (the union's V tiles)
 //   warp 11          idle
-// MMA order per union tile e: for each query tile that kept e: wait for its
-// P of the previous union tile (if it kept that one), issue its P V, issue S
-// for e; then for a query tile that did not keep e, issue its pending P V.
+// MMA order per union tile e: for each query tile that kept e: its P V of
+// the previous union tile (if it kept that one), then S for e; then for a
+// query tile that did not keep e, its pending P V.
 // So one query tile's softmax runs while the tensor core works for the
 // other, and the V slot of every union tile is released one step later, in
 // order (no ring can fill with tiles whose consumer is far ahead).
@@ -39,14 +39,14 @@ namespace {
 constexpr int BM = 128;               // rows per query tile
 constexpr int BN = 128;               // keys per tile
 constexpr int KST = 2, VST = 3;       // K and V ring stages
-constexpr float RESCALE_LOG2 = 8.0f;  // rescale O only when the max grows by > 2^8
+constexpr float OVERFLOW_SUM = 1.8446744e19f;  // 2^64: a tile's P sum above this moves the reference
 constexpr int POLY_PAIRS = 0x0;       // which pairs of every four run their exp2 on the FMA pipe
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_THREADS = 384;
 // Registers per thread after the split: softmax warpgroups (2 x 128 threads)
-// and the producer/MMA warpgroup (128 threads); 2*128*216 + 128*72 = 64,512
+// and the producer/MMA warpgroup (128 threads); 2*128*208 + 128*88 = 64,512
 // = the 384*168 the launch reserves.
-constexpr int REGS_SOFTMAX = 216, REGS_ROLES = 72;
+constexpr int REGS_SOFTMAX = 208, REGS_ROLES = 88;
 
 template <int D>
 struct PairLayout {
@@ -156,6 +156,32 @@ __device__ __forceinline__ void half_p(const uint32_t (&u)[64], int h, int klen,
   }
 }
 
+// Maximum of a row of S over its valid keys.
+template <bool FULL>
+__device__ __forceinline__ float row_max(const uint32_t (&u)[BN], int klen) {
+  const uint32_t (&u0)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&u[0]);
+  const uint32_t (&u1)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&u[64]);
+  return fmaxf(half_max<FULL>(u0, 0, klen), half_max<FULL>(u1, 1, klen));
+}
+
+// P = 2^(s*C - m) for a whole row as bf16 pairs (keys [0,64) in pk0, [64,128)
+// in pk1); returns the row sum of the fp32 values.
+template <bool FULL>
+__device__ __forceinline__ float row_p(const uint32_t (&u)[BN], int klen, uint64_t C2, float m, uint32_t (&pk0)[32],
+                                       uint32_t (&pk1)[32]) {
+  const uint32_t (&u0)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&u[0]);
+  const uint32_t (&u1)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&u[64]);
+  const uint64_t NM = f2(-m, -m);
+  uint64_t acc[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
+  half_p<FULL>(u0, 0, klen, C2, NM, acc, pk0);
+  half_p<FULL>(u1, 1, klen, C2, NM, acc, pk1);
+  float lo, hi;
+  f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
+  return lo + hi;
+}
+
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     sparse_attn_pair_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ CUtensorMap tmQ,
@@ -263,9 +289,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(BM, D, false, true);
-      const uint32_t aQ = smem_u32(smem + Lay::OFF_Q);
-      const uint32_t aK = smem_u32(smem + Lay::OFF_K);
-      const uint32_t aV = smem_u32(smem + Lay::OFF_V);
+      // Descriptors are built once; an operand's position inside a ring slot
+      // or a tile only adds (byte offset >> 4) to the start-address field,
+      // which never carries out of it for addresses below 256 KB.
+      const uint64_t dQ = sdesc_sw128(smem_u32(smem + Lay::OFF_Q), 16, 1024);
+      const uint64_t dK = sdesc_sw128(smem_u32(smem + Lay::OFF_K), 16, 1024);
+      const uint64_t dV = sdesc_sw128(smem_u32(smem + Lay::OFF_V), BN * 128, 1024);
       bool pend[2] = {false, false};
       int js[2] = {0, 0};  // S issued per query tile
       int prev_e = -1;
@@ -273,14 +302,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (ok) tc_fence_after();
       // P V for the tile kept at union position prev_e by query tile r
       auto issue_pv = [&](int r) -> bool {
+        const int vs = prev_e % VST;
         if (!mbar_wait(p_full + r, (js[r] - 1) & 1, abort_flag, g.dev_status)) return false;
-        if (!mbar_wait(v_full + prev_e % VST, (prev_e / VST) & 1, abort_flag, g.dev_status)) return false;
+        if (!mbar_wait(v_full + vs, (prev_e / VST) & 1, abort_flag, g.dev_status)) return false;
         tc_fence_after();
-        const uint32_t o_col = 2 * BN + r * D, s_col = r * BN;
+        const uint32_t o_addr = tmem + 2 * BN + r * D, p_addr = tmem + r * BN + 64;
+        const uint64_t dVs = dV + (uint64_t)(vs * (Lay::KB >> 4));
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ts(tmem + o_col, tmem + s_col + 64 + kk * 8,
-                       sdesc_sw128(aV + (prev_e % VST) * Lay::KB + kk * 2048, BN * 128, 1024), idesc_o,
+          umma_bf16_ts(o_addr, p_addr + kk * 8, dVs + (uint64_t)(kk * (2048 >> 4)), idesc_o,
                        (js[r] > 1 || kk > 0) ? 1u : 0u);
         umma_commit(pv_done + r);
         pend[r] = false;
@@ -299,11 +329,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int r = 0; r < 2; ++r) {
           if (!mem[r]) continue;
           if (pend[r] && !(ok = issue_pv(r))) break;
+          const uint64_t dQr = dQ + (uint64_t)(r * (Lay::QB >> 4)), dKs = dK + (uint64_t)(st * (Lay::KB >> 4));
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-            umma_bf16_ss(tmem + r * BN, sdesc_sw128(aQ + r * Lay::QB + off, 16, 1024),
-                         sdesc_sw128(aK + st * Lay::KB + off, 16, 1024), idesc_s, kk > 0);
+            const uint64_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+            umma_bf16_ss(tmem + r * BN, dQr + off, dKs + off, idesc_s, kk > 0);
           }
           umma_commit(s_full + r);
           js[r]++;
@@ -362,30 +392,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // the whole S row in registers: one TMEM load
       uint32_t u[BN];
       tmem_ld128(lane_addr + s_col, u);
-      float mx;
-      {
-        uint32_t (&u0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[0]);
-        uint32_t (&u1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[64]);
-        mx = full ? fmaxf(half_max<true>(u0, 0, klen), half_max<true>(u1, 1, klen))
-                  : fmaxf(half_max<false>(u0, 0, klen), half_max<false>(u1, 1, klen));
-      }
-      const float mx2 = mx * C;
-      if (j == 0) {
-        m = mx2;
-      } else {
-        const bool need = mx2 > m + RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, need)) {
+      if (j == 0) m = (full ? row_max<true>(u, klen) : row_max<false>(u, klen)) * C;
+      uint32_t pk0[32], pk1[32];
+      float ts = full ? row_p<true>(u, klen, C2, m, pk0, pk1) : row_p<false>(u, klen, C2, m, pk0, pk1);
+      // Later tiles are not max-reduced: P = 2^(s*C - m) may exceed 1 when a
+      // tile holds larger logits than the first one did, and fp32 / bf16 keep
+      // their relative precision at any magnitude, so the reference m only
+      // moves when the tile's sum nears the top of the range (rare). P is not
+      // stored yet, so S is still intact in TMEM for the exact recomputation.
+      const bool redo = !(ts <= OVERFLOW_SUM);
+      if (__any_sync(0xffffffffu, redo)) {
+        tmem_ld128(lane_addr + s_col, u);
+        const float mx2 = (full ? row_max<true>(u, klen) : row_max<false>(u, klen)) * C;
+        const float m_new = redo ? fmaxf(m, mx2) : m;
+        const float alpha = fast_exp2(m - m_new);
+        if (j > 0) {
           // O must hold P V of the previous tile before it is rescaled
           if (!__all_sync(0xffffffffu, mbar_wait(pv_done + r, (j - 1) & 1, abort_flag, g.dev_status))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const float alpha = need ? fast_exp2(m - mx2) : 1.0f;
-          if (need) {
-            l *= alpha;
-            m = mx2;
-          }
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -395,31 +422,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_st32(lane_addr + o_col + c * 32, o);
           }
         }
+        l *= alpha;
+        m = m_new;
+        ts = full ? row_p<true>(u, klen, C2, m, pk0, pk1) : row_p<false>(u, klen, C2, m, pk0, pk1);
       }
-      const uint64_t NM = f2(-m, -m);
-      uint64_t acc[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
-      // P (bf16 pairs) over columns [64,128) of S (all of S is in registers):
-      // keys [0,64) -> [64,96), keys [64,128) -> [96,128); both stores are
-      // asynchronous and waited for once, before P is announced
-      {
-        uint32_t (&u0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[0]);
-        uint32_t (&u1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&u[64]);
-        uint32_t pk0[32], pk1[32];
-        if (full) half_p<true>(u0, 0, klen, C2, NM, acc, pk0);
-        else half_p<false>(u0, 0, klen, C2, NM, acc, pk0);
-        tmem_st32_async(lane_addr + s_col + 64, pk0);
-        if (full) half_p<true>(u1, 1, klen, C2, NM, acc, pk1);
-        else half_p<false>(u1, 1, klen, C2, NM, acc, pk1);
-        tmem_st32_async(lane_addr + s_col + 96, pk1);
-        tmem_wait_st_keep(pk0, pk1);
-      }
-      {
-        float lo, hi;
-        f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
-        l += lo + hi;
-      }
+      // P (bf16 pairs) over columns [64,128) of S: keys [0,64) -> [64,96),
+      // keys [64,128) -> [96,128)
+      tmem_st32_async(lane_addr + s_col + 64, pk0);
+      tmem_st32_async(lane_addr + s_col + 96, pk1);
+      tmem_wait_st_keep(pk0, pk1);
+      l += ts;
       tc_fence_before();
       mbar_arrive(p_full + r);
     }

@@ -182,13 +182,18 @@ def test_topk_large_rows():
 
 # --------------------------------------------------------- sparse attention
 
-def _attention_case(w, k_override=None, dense=False, random_lists=True):
+def _attention_case(w, k_override=None, dense=False, random_lists=True, key_tile_gain=None):
     L = _layer(w)
     lays, perms, n_cap, nt_cap = oracle_geometry(w)
     q, k, v = _inputs(w)
     qp, _ = _permuted(L, w, q)
     kp, _ = _permuted(L, w, k)
     vp, _ = _permuted(L, w, v)
+    if key_tile_gain is not None:       # per key tile factor on K (and so on its logits)
+        for h in range(w.heads):
+            g = key_tile_gain(lays[h]["nt"])
+            for t, f in enumerate(g):
+                kp[:, h, t * w.tile:(t + 1) * w.tile] = (kp[:, h, t * w.tile:(t + 1) * w.tile].float() * f).bfloat16()
     ks = k_override or oracle_k(w, lays)
     k_cap = max(ks)
     idx = np.full((w.B, w.heads, nt_cap, k_cap), -1, np.int32)
@@ -235,6 +240,20 @@ def test_sparse_attention_k1_and_keep_all(name):
     lays, _, _, _ = oracle_geometry(w)
     _attention_case(w, k_override=[1] * w.heads)
     _attention_case(w, k_override=[l["nt"] for l in lays])
+
+
+@pytest.mark.parametrize("name", ["ragged-d128-t128", "batch2-d64-t128", "odd-d128-t64"])
+@pytest.mark.parametrize("order", ["growing", "shrinking"])
+def test_sparse_attention_wide_logit_range(name, order):
+    """Key tiles whose logits differ by hundreds of units: with `growing`, every
+    later kept tile out-scores the first one far beyond the fp32 exponent range
+    unless the running reference moves; with `shrinking`, later tiles
+    underflow against the first. Both must match the oracle's exact softmax."""
+    def gain(nt):
+        f = 1.0 + 6.0 * np.arange(nt)
+        return f if order == "growing" else f[::-1]
+    _attention_case(WL[name], key_tile_gain=gain)
+    _attention_case(WL[name], dense=True, key_tile_gain=gain)
 
 
 def test_sparse_attention_deterministic():
