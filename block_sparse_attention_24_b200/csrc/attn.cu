@@ -6,10 +6,10 @@
 //
 // Roles (224 threads):
 //   warps 0-3  softmax: thread r owns query row r = TMEM lane r. Reads a row
-//              of S from TMEM, keeps the running max / sum in fp32, writes P
+//              of S from TMEM, keeps the row reference and sum in fp32, writes P
 //              (bf16 pairs) back into the first half of the same TMEM
-//              columns, rescales O in TMEM when the max grows by more than
-//              2^8, and finally normalises O and stores it.
+//              columns, rescales O in TMEM on the rare block whose P sum
+//              nears the fp32 range, and finally normalises O and stores it.
 //   warp 4     K producer: TMA loads of Q once and of the selected K tiles
 //              into a 3-stage ring (128B-swizzled).
 //   warp 5     MMA issuer (one thread): S = Q K^T (A, B from shared memory)
@@ -35,8 +35,7 @@ namespace {
 constexpr int BM = 128;               // query rows per CTA
 constexpr int BN = 128;               // keys per block
 constexpr int KST = 3, VST = 3;       // K and V ring stages
-constexpr float RESCALE_LOG2 = 8.0f;  // rescale O only when the max grows by > 2^8
-constexpr int POLY_PAIRS = 0x8;       // which of the 4 pairs per 8-key chunk use the FMA-pipe exp2
+constexpr float OVERFLOW_SUM = 1.8446744e19f;  // 2^64: a block's P sum above this moves the reference
 constexpr uint32_t TMEM_COLS = 512;   // S0 [0,128), S1 [128,256), O [256, 256+D)
 constexpr int NUM_THREADS = 224;
 
@@ -247,22 +246,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int klen = tile_len(hg, g.T, kt);
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, ph, abort_flag, g.dev_status))) { ok = false; break; }
       tc_fence_after();
+      const bool full = klen == TILE;
       float sv[TILE];
-      {
+      // the row of S_j, masked past a padded key tile's valid prefix
+      auto load_s = [&]() {
         uint32_t u[TILE];
         if constexpr (TILE == 128) tmem_ld128(lane_addr + s * BN, u);
         else tmem_ld64(lane_addr + s * BN + sub * TILE, u);
 #pragma unroll
         for (int e = 0; e < TILE; ++e) sv[e] = __uint_as_float(u[e]);
-      }
-      const bool full = klen == TILE;
-      if (!full) {  // padded key tile: mask the columns past its valid prefix
+        if (!full) {
 #pragma unroll
-        for (int c = 0; c < TILE; ++c) sv[c] = c < klen ? sv[c] : -INFINITY;
-      }
+          for (int c = 0; c < TILE; ++c) sv[c] = c < klen ? sv[c] : -INFINITY;
+        }
+      };
       // row max: 8 independent 3-input max chains
-      float mx;
-      {
+      auto row_max = [&]() -> float {
         float pm[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) pm[i] = fmaxf(sv[i], sv[i + 8]);
@@ -270,14 +269,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 16; c < TILE; c += 16)
 #pragma unroll
           for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], sv[c + i], sv[c + 8 + i]);
-        mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-      }
-      const float mx2 = mx * C;
-      if (j == 0) {
-        m = mx2;
-      } else {
-        const bool need = mx2 > m + RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, need)) {
+        return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+      };
+      // P = 2^(s*C - mref) as bf16 pairs into pk, packed fp32x2 FMAs and
+      // MUFU ex2; returns the row sum.
+      uint32_t pk[64];  // the row of P: 128 keys as bf16 pairs
+      auto make_p = [&](float mref) -> float {
+        const uint64_t NM = f2(-mref, -mref);
+        uint64_t acc[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < 64; ++w) pk[w] = 0u;
+#pragma unroll
+        for (int q = 0; q < TILE / 8; ++q) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c0 = q * 8 + 2 * e;
+            const uint64_t x = f2_fma(f2(sv[c0], sv[c0 + 1]), C2, NM);
+            float x0, x1;
+            f2_split(x, x0, x1);
+            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            if (!full) {
+              p0 = c0 < klen ? p0 : 0.f;
+              p1 = c0 + 1 < klen ? p1 : 0.f;
+            }
+            acc[e] = f2_add(acc[e], f2(p0, p1));
+            if (NSUB == 1 || sub == 0) pk[c0 / 2] = pack_bf16x2_rn(p0, p1);
+            else pk[(TILE + c0) / 2] = pack_bf16x2_rn(p0, p1);
+          }
+        }
+        const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
+        float lo, hi;
+        f2_split(f2_add(a01, a23), lo, hi);
+        return lo + hi;
+      };
+      load_s();
+      // Only the first block of a row is max-reduced. Later blocks reuse its
+      // reference: P may exceed 1 when they hold larger logits, which fp32 and
+      // bf16 carry at full relative precision, so the reference moves only
+      // when a block's P sum nears the top of the range (rare); S_j is still
+      // in TMEM then (P is stored below), so the block is recomputed exactly.
+      if (j == 0) m = row_max() * C;
+      float rs = make_p(m);
+      const bool redo = !(rs <= OVERFLOW_SUM);
+      if (__any_sync(0xffffffffu, redo)) {
+        load_s();
+        const float mx2 = row_max() * C;
+        const float m_new = redo ? fmaxf(m, mx2) : m;
+        const float alpha = fast_exp2(m - m_new);
+        if (j > 0) {
           // O must hold PV_{j-1} before it is rescaled
           if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
                                                  g.dev_status))) {
@@ -285,11 +326,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const float alpha = need ? fast_exp2(m - mx2) : 1.0f;
-          if (need) {
-            l *= alpha;
-            m = mx2;
-          }
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t u[32];
@@ -299,46 +335,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_st32(lane_addr + 2 * BN + c * 32, u);
           }
         }
-      }
-      // P = 2^(s*C - m): packed fp32x2 FMAs; one pair in four on the FMA pipe
-      // (polynomial), the rest on MUFU; four packed partial row sums.
-      const uint64_t NM = f2(-m, -m);
-      uint64_t acc[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
-      uint32_t pk[64];  // the row of P: 128 keys as bf16 pairs
-#pragma unroll
-      for (int w = 0; w < 64; ++w) pk[w] = 0u;
-#pragma unroll
-      for (int q = 0; q < TILE / 8; ++q) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = q * 8 + 2 * e;
-          const uint64_t x = f2_fma(f2(sv[c0], sv[c0 + 1]), C2, NM);
-          float p0, p1;
-          if ((POLY_PAIRS >> e) & 1) {
-            f2_split(exp2_poly_f2(x), p0, p1);
-          } else {
-            float x0, x1;
-            f2_split(x, x0, x1);
-            p0 = fast_exp2(x0);
-            p1 = fast_exp2(x1);
-          }
-          if (!full) {
-            p0 = c0 < klen ? p0 : 0.f;
-            p1 = c0 + 1 < klen ? p1 : 0.f;
-          }
-          acc[e] = f2_add(acc[e], f2(p0, p1));
-          if (NSUB == 1 || sub == 0) pk[c0 / 2] = pack_bf16x2_rn(p0, p1);
-          else pk[(TILE + c0) / 2] = pack_bf16x2_rn(p0, p1);
-        }
-      }
-      float rs;
-      {
-        const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
-        float lo, hi;
-        f2_split(f2_add(a01, a23), lo, hi);
-        rs = lo + hi;
+        l *= alpha;
+        m = m_new;
+        rs = make_p(m);
       }
       l += rs;
       tmem_st64(lane_addr + s * BN, pk);  // P_j over the first half of S_j

@@ -40,7 +40,6 @@ constexpr int BM = 128;               // rows per query tile
 constexpr int BN = 128;               // keys per tile
 constexpr int KST = 2, VST = 3;       // K and V ring stages
 constexpr float OVERFLOW_SUM = 1.8446744e19f;  // 2^64: a tile's P sum above this moves the reference
-constexpr int POLY_PAIRS = 0x0;       // which pairs of every four run their exp2 on the FMA pipe
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_THREADS = 384;
 // Registers per thread after the split: softmax warpgroups (2 x 128 threads)
@@ -127,10 +126,9 @@ __device__ __forceinline__ float half_max(const uint32_t (&u)[64], int h, int kl
   return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
 }
 
-// P = 2^(s*C - m) for one 64-key half h of the row as 32 bf16 pairs, with
-// four packed partial row sums. Pairs selected by POLY_PAIRS (per group of
-// four) use the FMA-pipe polynomial, the rest MUFU ex2. Keys at or past
-// `klen` get P = 0 unless FULL.
+// P = 2^(s*C - m) for one 64-key half h of the row as 32 bf16 pairs (MUFU
+// ex2), with four packed partial row sums. Keys at or past `klen` get P = 0
+// unless FULL.
 template <bool FULL>
 __device__ __forceinline__ void half_p(const uint32_t (&u)[64], int h, int klen, uint64_t C2, uint64_t NM,
                                        uint64_t (&acc)[4], uint32_t (&pk)[32]) {
@@ -138,15 +136,9 @@ __device__ __forceinline__ void half_p(const uint32_t (&u)[64], int h, int klen,
   for (int w = 0; w < 32; ++w) {
     const int k0 = 64 * h + 2 * w;
     const uint64_t x = f2_fma(f2(__uint_as_float(u[2 * w]), __uint_as_float(u[2 * w + 1])), C2, NM);
-    float p0, p1;
-    if ((POLY_PAIRS >> (w & 3)) & 1) {
-      f2_split(exp2_poly_f2(x), p0, p1);
-    } else {
-      float x0, x1;
-      f2_split(x, x0, x1);
-      p0 = fast_exp2(x0);
-      p1 = fast_exp2(x1);
-    }
+    float x0, x1;
+    f2_split(x, x0, x1);
+    float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
     if (!FULL) {
       p0 = k0 < klen ? p0 : 0.f;
       p1 = k0 + 1 < klen ? p1 : 0.f;

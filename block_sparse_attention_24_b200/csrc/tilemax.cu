@@ -21,9 +21,10 @@ constexpr int KST = 3;                 // K ring stages
 constexpr uint32_t TMEM_COLS = 512;    // S buffers: row-block r, buffer b at (2r + b) * 128
 constexpr int NUM_THREADS = 384;
 // softmax warpgroups 216 registers, producer/MMA warpgroup 72:
-// 2*128*216 + 128*72 = 64,512 = the 384*168 the launch reserves
+// 2*128*216 + 128*72 = 64,512 = the 384*168 the launch reserves (208/88
+// removes the producer warps' few spills but measured 10% slower)
 constexpr int REGS_SOFTMAX = 216, REGS_ROLES = 72;
-constexpr int POLY_PAIRS = 0xA;        // pass 1: pairs 1 and 3 of every four use the FMA-pipe exp2
+constexpr float OVERFLOW_SUM = 1.8446744e19f;  // 2^64: a tile's exp sum above this moves the reference
 
 template <int D>
 struct MapLayout {
@@ -76,7 +77,7 @@ __device__ __forceinline__ float tile_max(const uint32_t (&u)[BN], int c0, int k
 }
 
 // Sum over columns [c0, c0+TILE) (the first `klen`, all when FULL) of
-// 2^(s*C - mnew); packed fp32x2 math, part of the exponentials on the FMA pipe.
+// 2^(s*C - mref); packed fp32x2 math, exponentials on MUFU.
 template <int TILE, bool FULL>
 __device__ __forceinline__ float tile_expsum(const uint32_t (&u)[BN], int c0, int klen, uint64_t C2, uint64_t NM) {
   uint64_t acc[4];
@@ -86,14 +87,9 @@ __device__ __forceinline__ float tile_expsum(const uint32_t (&u)[BN], int c0, in
   for (int w = 0; w < TILE / 2; ++w) {
     const int k0 = 2 * w;
     const uint64_t y = f2_fma(f2(__uint_as_float(u[c0 + k0]), __uint_as_float(u[c0 + k0 + 1])), C2, NM);
-    uint64_t p;
-    if ((POLY_PAIRS >> (w & 3)) & 1) {
-      p = exp2_poly_f2(y);
-    } else {
-      float y0, y1;
-      f2_split(y, y0, y1);
-      p = f2(fast_exp2(y0), fast_exp2(y1));
-    }
+    float y0, y1;
+    f2_split(y, y0, y1);
+    uint64_t p = f2(fast_exp2(y0), fast_exp2(y1));
     if (!FULL) {
       float p0, p1;
       f2_split(p, p0, p1);
@@ -274,17 +270,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kt = kb * NSUB + uu;
         const int klen = kt < nt ? tile_len(hg, g.T, kt) : 0;
         const bool full = klen >= TILE;
-        const float mx = full ? tile_max<TILE, true>(u, uu * TILE, klen) : tile_max<TILE, false>(u, uu * TILE, klen);
+        auto block_max = [&]() {
+          return full ? tile_max<TILE, true>(u, uu * TILE, klen) : tile_max<TILE, false>(u, uu * TILE, klen);
+        };
+        auto block_sum = [&](float mref) {
+          const uint64_t NM = f2(-mref, -mref);
+          return full ? tile_expsum<TILE, true>(u, uu * TILE, klen, C2, NM)
+                      : tile_expsum<TILE, false>(u, uu * TILE, klen, C2, NM);
+        };
         if (!pass2) {
+          // Only the row's first key tile is max-reduced; later tiles sum
+          // 2^(s*C - m) against that reference, which fp32 carries at full
+          // relative precision, and move it only when a tile's sum nears the
+          // top of the range (rare).
           if (klen > 0) {
-            const float mnew = fmaxf(m, mx * C);
-            const uint64_t NM = f2(-mnew, -mnew);
-            const float sum = full ? tile_expsum<TILE, true>(u, uu * TILE, klen, C2, NM)
-                                   : tile_expsum<TILE, false>(u, uu * TILE, klen, C2, NM);
-            l = l * fast_exp2(m - mnew) + sum;
-            m = mnew;
+            if (m == -INFINITY) m = block_max() * C;
+            float sum = block_sum(m);
+            if (!(sum <= OVERFLOW_SUM)) {
+              const float mnew = fmaxf(m, block_max() * C);
+              l *= fast_exp2(m - mnew);
+              m = mnew;
+              sum = block_sum(m);
+            }
+            l += sum;
           }
         } else {
+          const float mx = block_max();
           float v = (row_valid && klen > 0) ? fmaf(mx, C, -lse2) : -INFINITY;
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));

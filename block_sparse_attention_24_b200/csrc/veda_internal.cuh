@@ -353,28 +353,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair of x <= 8, on the FMA and integer pipes (no MUFU): x is
-// split into an integer j (rounded by adding 1.5*2^23) and f = x - j in
-// [-1/2, 1/2]; 2^f comes from a degree-3 polynomial fitted to 2^f on that
-// interval by Remez exchange for minimal relative error (max 7.5e-5), and j
-// is added to the exponent field. Inputs below -125 are clamped there.
-__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x) {
-  float x0, x1;
-  f2_split(x, x0, x1);
-  const uint64_t xc = f2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = f2_add(xc, f2(12582912.0f, 12582912.0f));
-  const uint64_t j = f2_add(t, f2(-12582912.0f, -12582912.0f));
-  const uint64_t f = f2_fma(j, f2(-1.0f, -1.0f), xc);
-  uint64_t p = f2_fma(f, f2(0.0551716685295105f, 0.0551716685295105f), f2(0.2426111251115799f, 0.2426111251115799f));
-  p = f2_fma(p, f, f2(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2(0.9999280571937561f, 0.9999280571937561f));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  return f2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
-            __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

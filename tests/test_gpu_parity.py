@@ -294,11 +294,31 @@ def test_tilemap_lse_kl(name):
     w = WL[name]
     if w.B != 1:
         pytest.skip("tile map is defined for B == 1 layers")
+    _tilemap_case(w)
+
+
+@pytest.mark.parametrize("name", ["ragged-d128-t128", "odd-d128-t64", "d64-t64-padded"])
+@pytest.mark.parametrize("order", ["growing", "shrinking"])
+def test_tilemap_wide_logit_range(name, order):
+    """Key tiles whose logits differ by hundreds of units (as in the attention
+    case): the row log-sum-exp must move its reference when a later key tile
+    out-scores the first one beyond the fp32 exponent range."""
+    def gain(nt):
+        f = 1.0 + 6.0 * np.arange(nt)
+        return f if order == "growing" else f[::-1]
+    _tilemap_case(WL[name], key_tile_gain=gain)
+
+
+def _tilemap_case(w, key_tile_gain=None):
     L = _layer(w)
     lays, perms, n_cap, nt_cap = oracle_geometry(w)
     q, k, _ = _inputs(w)
     qp, _ = _permuted(L, w, q)
     kp, _ = _permuted(L, w, k)
+    if key_tile_gain is not None:
+        for h in range(w.heads):
+            for t, f in enumerate(key_tile_gain(lays[h]["nt"])):
+                kp[:, h, t * w.tile:(t + 1) * w.tile] = (kp[:, h, t * w.tile:(t + 1) * w.tile].float() * f).bfloat16()
     heads = list(range(w.heads))
     n_rows = min(l["nt"] for l in lays)
     rows = np.stack([np.sort(np.random.default_rng(h).choice(lays[h]["nt"], n_rows, replace=False))
