@@ -38,7 +38,7 @@ import synth  # noqa: E402
 METRIC = "block-sparse attn ms/layer & effective TFLOP/s at 90% sparsity vs dense path"
 UNIT = "TFLOP/s"
 MAP_ROWS = 120          # query tiles per tile-map head (10% of 1200: sparse supervision)
-KERNELS_PER_STEP = 13   # 3 permute, 2 TripPool, MLP + score GEMM, top-k, attention, unpermute, map, KL rows, KL mean
+KERNELS_PER_STEP = 11   # 2 permute+TripPool, permute V, MLP + score GEMM, top-k, attention, unpermute, map, KL rows, KL mean
 
 
 # ------------------------------------------------------------------ ranks
@@ -294,16 +294,14 @@ def run_ours(args, world, rank, local):
 
 
 def stage_breakdown(V, L, layer, q, k, v, stream):
-    names = ["permute_qkv", "trippool_qk", "tile_scores", "topk"]
+    names = ["permute_trippool_qk", "permute_v", "tile_scores", "topk"]
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
     w = layer.w
     ev[0].record(stream)
-    V.veda_permute(L, q, layer.qp, layer.perm)
-    V.veda_permute(L, k, layer.kp)
-    V.veda_permute(L, v, layer.vp)
+    V.veda_permute_trippool(L, q, layer.qp, layer.dq, layer.perm)
+    V.veda_permute_trippool(L, k, layer.kp, layer.dk)
     ev[1].record(stream)
-    V.veda_trippool(L, layer.qp, layer.dq)
-    V.veda_trippool(L, layer.kp, layer.dk)
+    V.veda_permute(L, v, layer.vp)
     ev[2].record(stream)
     V.veda_tile_scores(L, layer.dq, layer.dk, w["w1q"], w["b1q"], w["w2q"], w["b2q"], w["w1k"], w["b1k"], w["w2k"],
                        w["b2k"], layer.hidden, layer.out_dim, layer.score_scale, layer.scores, layer.emb_ws)
@@ -385,10 +383,11 @@ def frontend_bandwidth(L, layer, stage_ms, unperm_ms, hbm_gbs):
     row = d * 2
     nt_sum = sum(L.nt) * B
     byts = {
-        # read every original row, write every permuted row (incl. padding), x3 tensors
-        "permute_qkv": 3 * (valid * row + B * Hh * L.n_cap * row),
-        # read the valid rows of Qp and Kp, write [avg|max|min] fp32 per tile
-        "trippool_qk": 2 * (valid * row + nt_sum * 3 * d * 4),
+        # Q and K: read every original row, write every permuted row (incl.
+        # padding) and [avg|max|min] fp32 per tile
+        "permute_trippool_qk": 2 * (valid * row + B * Hh * L.n_cap * row + nt_sum * 3 * d * 4),
+        # V: read every original row, write every permuted row
+        "permute_v": valid * row + B * Hh * L.n_cap * row,
         # read the scores, write index lists and the dense mask
         "topk": B * Hh * L.nt_cap * L.nt_cap * 4 + B * Hh * L.nt_cap * (layer.k_cap * 4 + L.nt_cap),
     }

@@ -25,7 +25,7 @@ VEDA_ERR_CUDA = -3
 VEDA_ERR_TIMEOUT = -4
 VEDA_ERR_BAD_INDEX = -5
 
-EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
+EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
             "veda_topk_mask", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
             "veda_selftest_wait_timeout", "veda_last_error")
@@ -63,6 +63,7 @@ _LP = ctypes.POINTER(_Layer)
 _lib.veda_layout.argtypes = [_LP, _P, _P, _P, _P]
 _lib.veda_permute.argtypes = [_LP, _P, _P, _P, ctypes.c_int, _P]
 _lib.veda_trippool.argtypes = [_LP, _P, _P, _P]
+_lib.veda_permute_trippool.argtypes = [_LP, _P, _P, _P, _P, _P]
 _lib.veda_tile_scores.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _P, _P]
 _lib.veda_tile_scores_noalloc.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _P]
 _lib.veda_tile_scores_ws_bytes.argtypes = [_LP, _I]
@@ -146,6 +147,11 @@ def veda_permute(layer: Layer, x: torch.Tensor, xp: torch.Tensor, perm: Optional
 
 def veda_trippool(layer: Layer, xp: torch.Tensor, desc: torch.Tensor, stream=None):
     _check(_lib.veda_trippool(layer.ref, _ptr(xp), _ptr(desc), _stream(stream)))
+
+
+def veda_permute_trippool(layer: Layer, x: torch.Tensor, xp: torch.Tensor, desc: torch.Tensor,
+                          perm: Optional[torch.Tensor] = None, stream=None):
+    _check(_lib.veda_permute_trippool(layer.ref, _ptr(x), _ptr(xp), _ptr(perm), _ptr(desc), _stream(stream)))
 
 
 def veda_tile_scores_ws_bytes(layer: Layer, out_dim: int) -> int:

@@ -164,6 +164,17 @@ int veda_trippool(const veda_layer* L, const void* xp, float* desc, cudaStream_t
   return after_launch(veda::launch_trippool(g, xp, desc, stream), "veda_trippool");
 }
 
+int veda_permute_trippool(const veda_layer* L, const void* x, void* xp, int32_t* perm, float* desc,
+                          cudaStream_t stream) {
+  veda::LayerGeom g;
+  VEDA_TRY(build_geom(L, &g));
+  VEDA_TRY(check_ptr(x, "x"));
+  VEDA_TRY(check_ptr(xp, "xp"));
+  VEDA_TRY(check_ptr(desc, "desc"));
+  if (perm) VEDA_TRY(check_ptr(perm, "perm"));
+  return after_launch(veda::launch_permute_pool(g, x, xp, perm, desc, stream), "veda_permute_trippool");
+}
+
 size_t veda_tile_scores_ws_bytes(const veda_layer* L, int32_t out_dim) {
   veda::LayerGeom g;
   if (build_geom(L, &g) != VEDA_OK || out_dim < 1) return 0;

@@ -1,7 +1,7 @@
 """One Veda attention layer on the device: the C-ABI calls of the hot path in
 order, over buffers allocated once.
 
-    permute(Q, K, V) -> TripPool(Qp, Kp) -> tile scores -> top-k mask
+    permute + TripPool (Q, K), permute (V) -> tile scores -> top-k mask
       -> tile-skipping sparse attention -> inverse permute
     (+ distillation rows: full-attention tile map on selected heads and query
        tiles, row-wise KL against the predicted scores)
@@ -17,8 +17,8 @@ from typing import Dict, List, Optional, Sequence
 
 import torch
 
-from . import (Layer, veda_full_attn_tilemax, veda_permute, veda_sparse_attn, veda_tile_scores,
-               veda_tile_scores_ws_bytes, veda_topk_mask, veda_trippool)
+from . import (Layer, veda_full_attn_tilemax, veda_permute, veda_permute_trippool, veda_sparse_attn,
+               veda_tile_scores, veda_tile_scores_ws_bytes, veda_topk_mask)
 
 
 def k_from_keep(keep: float, nt: int) -> int:
@@ -34,8 +34,8 @@ class MapRequest:
 
 
 class VedaLayer:
-    STAGES = ("permute_q", "permute_k", "permute_v", "trippool_q", "trippool_k", "tile_scores", "topk",
-              "sparse_attn", "unpermute", "tilemap_kl")
+    STAGES = ("permute_trippool_q", "permute_trippool_k", "permute_v", "tile_scores", "topk", "sparse_attn",
+              "unpermute", "tilemap_kl")
 
     def __init__(self, layer: Layer, keep: Optional[float], weights: Dict[str, torch.Tensor], score_scale: float,
                  device, k: Optional[Sequence[int]] = None, maps: Optional[MapRequest] = None):
@@ -94,11 +94,10 @@ class VedaLayer:
     # -- the hot path -------------------------------------------------------
     def front(self, q, k, v, stream=None):
         L = self.L
-        veda_permute(L, q, self.qp, self.perm, stream=stream)
-        veda_permute(L, k, self.kp, stream=stream)
+        # Q and K: permutation and TripPool in one pass; V: permutation only
+        veda_permute_trippool(L, q, self.qp, self.dq, self.perm, stream=stream)
+        veda_permute_trippool(L, k, self.kp, self.dk, stream=stream)
         veda_permute(L, v, self.vp, stream=stream)
-        veda_trippool(L, self.qp, self.dq, stream=stream)
-        veda_trippool(L, self.kp, self.dk, stream=stream)
         w = self.w
         veda_tile_scores(L, self.dq, self.dk, w["w1q"], w["b1q"], w["w2q"], w["b2q"], w["w1k"], w["b1k"], w["w2k"],
                          w["b2k"], self.hidden, self.out_dim, self.score_scale, self.scores, self.emb_ws,

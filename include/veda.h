@@ -95,6 +95,16 @@ int veda_permute(const veda_layer* L, const void* x, void* xp, int32_t* perm,
  * xp [B,heads,n_cap,d] bf16 -> desc [B,heads,nt_cap,3d] fp32. */
 int veda_trippool(const veda_layer* L, const void* xp, float* desc, cudaStream_t stream);
 
+/* The forward permutation and TripPool in one pass (Veda summary 2.1 and
+ * 2.2; the pages name tighter kernel fusion as future work): x -> xp and
+ * perm exactly as veda_permute(..., inverse = 0), and desc [B,heads,nt_cap,
+ * 3d] fp32 as veda_trippool would compute from xp, without reading xp back.
+ * max/min are bit-identical to veda_trippool; the mean sums the same values
+ * in another order (fp32 rounding). `perm` may be NULL. All pointers are
+ * caller-owned device memory, 16-byte aligned. */
+int veda_permute_trippool(const veda_layer* L, const void* x, void* xp, int32_t* perm, float* desc,
+                          cudaStream_t stream);
+
 /* Head-specific MLP estimator and tile scores (Veda summary 2.1,
  * Head-Specific Projections): per head h,
  *   q_i = W2q^T GELU(W1q^T dq_i + b1q) + b2q,  k_j likewise with the k weights,

@@ -75,6 +75,11 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     assert rc == V.VEDA_ERR_INVALID_ARG and "NULL" in V.veda_last_error()
     rc = lib.veda_permute(L.ref, ctypes.c_void_p(0x1008), ctypes.c_void_p(0x2000), None, 0, None)
     assert rc == V.VEDA_ERR_INVALID_ARG and "aligned" in V.veda_last_error()
+    rc = lib.veda_permute_trippool(L.ref, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), None, None, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "desc" in V.veda_last_error()
+    rc = lib.veda_permute_trippool(L.ref, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3004),
+                                   ctypes.c_void_p(0x4000), None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "perm" in V.veda_last_error()
     k = (ctypes.c_int32 * 2)(5, 1)      # k > nt for head 0
     rc = lib.veda_topk_mask(L.ref, ctypes.c_void_p(0x1000), k, 8, ctypes.c_void_p(0x2000), None, None)
     assert rc == V.VEDA_ERR_INVALID_ARG and "k=5" in V.veda_last_error()

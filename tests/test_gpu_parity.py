@@ -103,6 +103,44 @@ def test_trippool(name):
             assert not got[b, h, nt:].any()
 
 
+@pytest.mark.parametrize("name", list(WL))
+def test_permute_trippool_fused(name):
+    """The fused call against the oracle (permutation and max/min bit-exact,
+    mean within fp32 rounding) and against the two unfused calls."""
+    w = WL[name]
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, _, _ = _inputs(w)
+    xp = torch.full((w.B, w.heads, n_cap, w.d), 7.0, dtype=torch.bfloat16, device=DEV)   # poisoned
+    perm = torch.full((w.heads, n_cap), 12345, dtype=torch.int32, device=DEV)
+    desc = torch.full((w.B, w.heads, nt_cap, 3 * w.d), 7.0, dtype=torch.float32, device=DEV)
+    V.veda_permute_trippool(L, q, xp, desc, perm)
+    V.veda_check_status(L)
+    pg = perm.cpu().numpy()
+    for h in range(w.heads):
+        assert np.array_equal(pg[h, :len(perms[h])], perms[h])
+        assert (pg[h, len(perms[h]):] == -1).all()
+    assert np.array_equal(f64(xp), O.permute(f64(q), perms, n_cap))
+    got, d = desc.cpu().double().numpy(), w.d
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt = lays[h]["nt"]
+            ref = O.trippool(f64(xp)[b, h], lays[h]["lens"], w.tile)
+            np.testing.assert_allclose(got[b, h, :nt, :d], ref[:, :d], rtol=1e-6, atol=1e-6)
+            assert np.array_equal(got[b, h, :nt, d:], ref[:, d:])
+            assert not got[b, h, nt:].any()
+    # same max/min as the unfused TripPool; the permuted tensor identical
+    xp2, _ = _permuted(L, w, q)
+    desc2 = torch.empty_like(desc)
+    V.veda_trippool(L, xp2, desc2)
+    torch.cuda.synchronize()
+    assert torch.equal(xp, xp2)
+    assert torch.equal(desc[..., d:], desc2[..., d:])
+    # no perm map requested
+    V.veda_permute_trippool(L, q, xp, desc)
+    V.veda_check_status(L)
+
+
 # ------------------------------------------------------------- tile scores
 
 @pytest.mark.parametrize("name", list(WL))
