@@ -390,6 +390,7 @@ def frontend_bandwidth(L, layer, stage_ms, unperm_ms, hbm_gbs):
         "permute_v": valid * row + B * Hh * L.n_cap * row,
         # read the scores, write index lists and the dense mask
         "topk": B * Hh * L.nt_cap * L.nt_cap * 4 + B * Hh * L.nt_cap * (layer.k_cap * 4 + L.nt_cap),
+
     }
     out = {}
     for k, b in byts.items():

@@ -27,7 +27,7 @@ VEDA_ERR_BAD_INDEX = -5
 
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
-            "veda_topk_mask", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
+            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
             "veda_selftest_wait_timeout", "veda_last_error")
 
 
@@ -69,6 +69,7 @@ _lib.veda_tile_scores_noalloc.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _P
 _lib.veda_tile_scores_ws_bytes.argtypes = [_LP, _I]
 _lib.veda_tile_scores_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_topk_mask.argtypes = [_LP, _P, _P, _I, _P, _P, _P]
+_lib.veda_tile_scores_topk.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _P, _P, _P, _P]
 _lib.veda_sparse_attn.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
 _lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P, _P, _P, _P, _P]
 _lib.veda_check_status.argtypes = [_LP, _P]
@@ -183,6 +184,14 @@ def veda_topk_mask(layer: Layer, scores: torch.Tensor, k: Sequence[int], k_cap: 
                    mask: Optional[torch.Tensor] = None, stream=None):
     _check(_lib.veda_topk_mask(layer.ref, _ptr(scores), _host_i32(k), int(k_cap), _ptr(idx), _ptr(mask),
                                _stream(stream)))
+
+
+def veda_tile_scores_topk(layer: Layer, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden: int, out_dim: int,
+                          scale: float, k: Sequence[int], k_cap: int, idx: torch.Tensor, emb_ws: torch.Tensor,
+                          mask: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None, stream=None):
+    _check(_lib.veda_tile_scores_topk(layer.ref, *[_ptr(t) for t in (dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k)],
+                                      hidden, out_dim, float(scale), _host_i32(k), int(k_cap), _ptr(idx), _ptr(mask),
+                                      _ptr(scores), _ptr(emb_ws), _stream(stream)))
 
 
 def veda_sparse_attn(layer: Layer, qp, kp, vp, idx: Optional[torch.Tensor], k: Optional[Sequence[int]], k_cap: int,

@@ -216,6 +216,37 @@ int veda_topk_mask(const veda_layer* L, const float* scores, const int32_t* k, i
   return after_launch(veda::launch_topk(g, scores, k_cap, idx, mask, stream), "veda_topk_mask");
 }
 
+int veda_tile_scores_topk(const veda_layer* L, const float* dq, const float* dk, const float* w1q, const float* b1q,
+                          const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
+                          const float* b2k, int32_t hidden, int32_t out_dim, float scale, const int32_t* k,
+                          int32_t k_cap, int32_t* idx, uint8_t* mask, float* scores, float* emb_ws,
+                          cudaStream_t stream) {
+  veda::LayerGeom g;
+  VEDA_TRY(build_geom(L, &g));
+  const void* ptrs[] = {dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, idx, emb_ws};
+  const char* names[] = {"dq", "dk", "w1q", "b1q", "w2q", "b2q", "w1k", "b1k", "w2k", "b2k", "idx", "emb_ws"};
+  for (int i = 0; i < 12; ++i) VEDA_TRY(check_ptr(ptrs[i], names[i]));
+  if (mask) VEDA_TRY(check_ptr(mask, "mask"));
+  if (scores) VEDA_TRY(check_ptr(scores, "scores"));
+  if (hidden < 4 || hidden > 256 || hidden % 4)
+    return fail(VEDA_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 4 in [4, 256]", hidden);
+  if (out_dim < 4 || out_dim > 128 || out_dim % 4)
+    return fail(VEDA_ERR_UNSUPPORTED, "out_dim=%d must be a multiple of 4 in [4, 128]", out_dim);
+  if (!k) return fail(VEDA_ERR_INVALID_ARG, "k is NULL");
+  if (k_cap < 1) return fail(VEDA_ERR_INVALID_ARG, "k_cap=%d must be >= 1", k_cap);
+  for (int h = 0; h < g.heads; ++h) {
+    if (k[h] < 1 || k[h] > g.h[h].nt || k[h] > k_cap)
+      return fail(VEDA_ERR_INVALID_ARG, "head %d: k=%d outside [1, min(nt=%d, k_cap=%d)]", h, k[h], g.h[h].nt, k_cap);
+    g.h[h].k = k[h];
+  }
+  if ((size_t)g.nt_cap * 4 + (size_t)out_dim * 4 + 8 * 256 * 4 > 200 * 1024)
+    return fail(VEDA_ERR_UNSUPPORTED, "nt_cap=%d: a score row does not fit the fused kernel's shared memory", g.nt_cap);
+  cudaError_t e = veda::launch_mlp(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws, stream);
+  if (e != cudaSuccess) return after_launch(e, "veda_tile_scores_topk");
+  return after_launch(veda::launch_score_topk(g, emb_ws, out_dim, scale, k_cap, idx, mask, scores, stream),
+                      "veda_tile_scores_topk");
+}
+
 int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const void* vp, const int32_t* idx,
                      const int32_t* k, int32_t k_cap, float scale, void* op, float* lse, cudaStream_t stream) {
   veda::LayerGeom g;

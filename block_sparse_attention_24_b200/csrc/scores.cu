@@ -186,16 +186,22 @@ __global__ void __launch_bounds__(256) score_gemm_kernel(const __grid_constant__
 
 }  // namespace
 
-cudaError_t launch_tile_scores(const LayerGeom& g, const float* dq, const float* dk, const float* w1q,
-                               const float* b1q, const float* w2q, const float* b2q, const float* w1k,
-                               const float* b1k, const float* w2k, const float* b2k, int hidden, int out_dim,
-                               float scale, float* scores, float* emb_ws, cudaStream_t s) {
+cudaError_t launch_mlp(const LayerGeom& g, const float* dq, const float* dk, const float* w1q, const float* b1q,
+                       const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
+                       const float* b2k, int hidden, int out_dim, float* emb_ws, cudaStream_t s) {
   const size_t smem = (size_t)MLP_ROWS * (3 * g.d + hidden) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 g1((g.nt_cap + MLP_ROWS - 1) / MLP_ROWS, g.heads, g.B * 2);
   mlp_kernel<<<g1, 128, smem, s>>>(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws);
-  e = cudaGetLastError();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_scores(const LayerGeom& g, const float* dq, const float* dk, const float* w1q,
+                               const float* b1q, const float* w2q, const float* b2q, const float* w1k,
+                               const float* b1k, const float* w2k, const float* b2k, int hidden, int out_dim,
+                               float scale, float* scores, float* emb_ws, cudaStream_t s) {
+  cudaError_t e = launch_mlp(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws, s);
   if (e != cudaSuccess) return e;
   const int nb = (g.nt_cap + 63) / 64;
   const dim3 g2(nb, nb, g.heads * g.B);

@@ -8,6 +8,7 @@
 // every key > T and the lowest-index keys == T, so exact ties go to the lower
 // tile index and the output list comes out ascending without a sort.
 // Histogram updates are warp-aggregated (__match_any_sync) shared atomics.
+// The same selection also runs inside the fused scores + top-k kernel.
 #include "veda_internal.cuh"
 
 namespace veda {
@@ -21,32 +22,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_constant__ LayerGeom g,
-                                                               const float* __restrict__ scores, int k_cap,
-                                                               int32_t* __restrict__ idx, uint8_t* __restrict__ mask) {
-  extern __shared__ uint32_t sm_u32[];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  uint32_t* keys = sm_u32 + warp * (g.nt_cap + 256);
-  uint32_t* hist = keys + g.nt_cap;
-  const long long rows = (long long)g.B * g.heads * g.nt_cap;
-  const long long row = (long long)blockIdx.x * TOPK_WARPS + warp;
-  if (row >= rows) return;
-  const int a = (int)(row % g.nt_cap);
-  const int h = (int)((row / g.nt_cap) % g.heads);
-  const int nt = g.h[h].nt;
-  const int k = g.h[h].k;
-  int32_t* idx_row = idx + row * k_cap;
-  uint8_t* mask_row = mask ? mask + row * g.nt_cap : nullptr;
-  if (a >= nt) {
-    for (int p = lane; p < k_cap; p += 32) idx_row[p] = -1;
-    if (mask_row)
-      for (int c = lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
-    return;
-  }
-  const float* srow = scores + row * g.nt_cap;
-  for (int c = lane; c < nt; c += 32) keys[c] = order_key(__ldg(srow + c));
-  __syncwarp();
-
+// Selection on one row staged as order keys in shared memory (warp-wide):
+// writes the k kept column indices ascending (-1 beyond k, up to k_cap) and
+// the 0/1 mask over nt_cap columns (when mask_row is not NULL). `hist` is 256
+// words of this warp's shared memory.
+__device__ __forceinline__ void warp_select_row(const uint32_t* keys, uint32_t* hist, int nt, int k, int k_cap,
+                                                int nt_cap, int32_t* idx_row, uint8_t* mask_row, int lane) {
   uint32_t prefix = 0u, pmask = 0u;
   int remaining = k;
 #pragma unroll 1
@@ -122,7 +103,117 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_cons
   }
   for (int p = k + lane; p < k_cap; p += 32) idx_row[p] = -1;
   if (mask_row)
-    for (int c = nt + lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
+    for (int c = nt + lane; c < nt_cap; c += 32) mask_row[c] = 0;
+}
+
+__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_constant__ LayerGeom g,
+                                                               const float* __restrict__ scores, int k_cap,
+                                                               int32_t* __restrict__ idx, uint8_t* __restrict__ mask) {
+  extern __shared__ uint32_t sm_u32[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint32_t* keys = sm_u32 + warp * (g.nt_cap + 256);
+  uint32_t* hist = keys + g.nt_cap;
+  const long long rows = (long long)g.B * g.heads * g.nt_cap;
+  const long long row = (long long)blockIdx.x * TOPK_WARPS + warp;
+  if (row >= rows) return;
+  const int a = (int)(row % g.nt_cap);
+  const int h = (int)((row / g.nt_cap) % g.heads);
+  const int nt = g.h[h].nt;
+  const int k = g.h[h].k;
+  int32_t* idx_row = idx + row * k_cap;
+  uint8_t* mask_row = mask ? mask + row * g.nt_cap : nullptr;
+  if (a >= nt) {
+    for (int p = lane; p < k_cap; p += 32) idx_row[p] = -1;
+    if (mask_row)
+      for (int c = lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
+    return;
+  }
+  const float* srow = scores + row * g.nt_cap;
+  for (int c = lane; c < nt; c += 32) keys[c] = order_key(__ldg(srow + c));
+  __syncwarp();
+
+  warp_select_row(keys, hist, nt, k, k_cap, g.nt_cap, idx_row, mask_row, lane);
+}
+
+// Tile scores and top-k in one pass (Veda summary 2.1; the pages name
+// tighter kernel fusion as future work). A CTA takes R query tiles of one
+// head, computes their whole score rows scale * q_i . k_j into shared memory
+// with the same fma order as the score GEMM kernel (so scores and selections
+// are bit-identical to the unfused path) and selects from there: the score
+// matrix reaches HBM only when the caller asks for it. Measured 1.07 ms
+// against 0.85 ms for the score GEMM plus top-k kernels on the 153,600-token
+// layer (the per-thread dot products with broadcast shared-memory operands
+// cannot match the register-tiled GEMM), so the layer uses the unfused pair.
+constexpr int ST_THREADS = 256, ST_WARPS = ST_THREADS / 32, ST_RMAX = 8;
+
+__global__ void __launch_bounds__(ST_THREADS) score_topk_kernel(const __grid_constant__ LayerGeom g,
+                                                                const float* __restrict__ emb, int out_dim,
+                                                                float scale, int R, int k_cap,
+                                                                int32_t* __restrict__ idx,
+                                                                uint8_t* __restrict__ mask,
+                                                                float* __restrict__ scores) {
+  extern __shared__ uint32_t sm_u32[];
+  float* qs = reinterpret_cast<float*>(sm_u32);                  // [R][out_dim], 16-byte rows (out_dim % 4 == 0)
+  uint32_t* hist = sm_u32 + R * out_dim;                         // [ST_WARPS][256]
+  uint32_t* keys = hist + ST_WARPS * 256;                        // [R][nt_cap] order keys
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int i0 = blockIdx.x * R;
+  const HeadGeom& hg = g.h[h];
+  const int nt = hg.nt;
+  const long long bh = (long long)b * g.heads + h;
+  const float* Q = emb + bh * g.nt_cap * out_dim;
+  const float* K = emb + ((long long)g.B * g.heads + bh) * g.nt_cap * out_dim;
+  for (int t = threadIdx.x; t < R * out_dim; t += ST_THREADS) {
+    const int r = t / out_dim;
+    qs[t] = i0 + r < nt ? Q[(long long)i0 * out_dim + t] : 0.f;
+  }
+  __syncthreads();
+  // one key tile per thread at a time, all R rows against it
+  for (int j = threadIdx.x; j < g.nt_cap; j += ST_THREADS) {
+    float acc[ST_RMAX];
+#pragma unroll
+    for (int r = 0; r < ST_RMAX; ++r) acc[r] = 0.f;
+    if (j < nt) {
+      const float4* kr = reinterpret_cast<const float4*>(K + (long long)j * out_dim);
+      for (int e4 = 0; e4 < out_dim / 4; ++e4) {
+        const float4 kv = __ldg(kr + e4);
+#pragma unroll
+        for (int r = 0; r < ST_RMAX; ++r) {
+          if (r < R) {
+            const float4 qv = *reinterpret_cast<const float4*>(qs + r * out_dim + 4 * e4);
+            acc[r] = fmaf(qv.x, kv.x, acc[r]);
+            acc[r] = fmaf(qv.y, kv.y, acc[r]);
+            acc[r] = fmaf(qv.z, kv.z, acc[r]);
+            acc[r] = fmaf(qv.w, kv.w, acc[r]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < ST_RMAX; ++r) {
+      if (r < R) {
+        const int i = i0 + r;
+        const float sc = (i < nt && j < nt) ? acc[r] * scale : 0.f;
+        keys[r * g.nt_cap + j] = order_key(sc);
+        if (scores && i < g.nt_cap) scores[(bh * g.nt_cap + i) * g.nt_cap + j] = sc;
+      }
+    }
+  }
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int r = warp; r < R; r += ST_WARPS) {
+    const int i = i0 + r;
+    if (i >= g.nt_cap) break;
+    int32_t* idx_row = idx + (bh * g.nt_cap + i) * k_cap;
+    uint8_t* mask_row = mask ? mask + (bh * g.nt_cap + i) * g.nt_cap : nullptr;
+    if (i >= nt) {  // query tile beyond this head's tiles
+      for (int p = lane; p < k_cap; p += 32) idx_row[p] = -1;
+      if (mask_row)
+        for (int c = lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
+      continue;
+    }
+    warp_select_row(keys + r * g.nt_cap, hist + warp * 256, nt, hg.k, k_cap, g.nt_cap, idx_row, mask_row, lane);
+  }
 }
 
 }  // namespace
@@ -136,6 +227,25 @@ cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int3
   const long long blocks = (rows + TOPK_WARPS - 1) / TOPK_WARPS;
   if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
   topk_kernel<<<(unsigned)blocks, TOPK_WARPS * 32, smem, s>>>(g, scores, k_cap, idx, mask);
+  return cudaGetLastError();
+}
+
+// Rows per CTA: as many as fit 200 KB of shared memory with the order keys
+// of whole rows, at most 8 (4 and 16 measured slower on the 153,600-token
+// layer: fewer rows re-read the key embeddings more often, more rows leave
+// too few CTAs per SM for the latency-bound selection).
+cudaError_t launch_score_topk(const LayerGeom& g, const float* emb_ws, int out_dim, float scale, int k_cap,
+                              int32_t* idx, uint8_t* mask, float* scores, cudaStream_t s) {
+  const size_t fixed = (size_t)ST_WARPS * 256 * 4;
+  const size_t per_row = (size_t)g.nt_cap * 4 + (size_t)out_dim * 4;
+  int R = (int)((200 * 1024 - fixed) / per_row);
+  R = R > ST_RMAX ? ST_RMAX : R;
+  if (R < 1) return cudaErrorInvalidValue;
+  const size_t smem = fixed + (size_t)R * per_row;
+  cudaError_t e = cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((g.nt_cap + R - 1) / R, g.heads, g.B);
+  score_topk_kernel<<<grid, ST_THREADS, smem, s>>>(g, emb_ws, out_dim, scale, R, k_cap, idx, mask, scores);
   return cudaGetLastError();
 }
 

@@ -379,6 +379,11 @@ cudaError_t launch_permute(const LayerGeom& g, const void* x, void* xp, int32_t*
 cudaError_t launch_trippool(const LayerGeom& g, const void* xp, float* desc, cudaStream_t s);
 cudaError_t launch_permute_pool(const LayerGeom& g, const void* x, void* xp, int32_t* perm, float* desc,
                                 cudaStream_t s);
+cudaError_t launch_mlp(const LayerGeom& g, const float* dq, const float* dk, const float* w1q, const float* b1q,
+                       const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
+                       const float* b2k, int hidden, int out_dim, float* emb_ws, cudaStream_t s);
+cudaError_t launch_score_topk(const LayerGeom& g, const float* emb_ws, int out_dim, float scale, int k_cap,
+                              int32_t* idx, uint8_t* mask, float* scores, cudaStream_t s);
 cudaError_t launch_tile_scores(const LayerGeom& g, const float* dq, const float* dk, const float* w1q,
                                const float* b1q, const float* w2q, const float* b2q, const float* w1k,
                                const float* b1k, const float* w2k, const float* b2k, int hidden, int out_dim,

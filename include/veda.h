@@ -146,6 +146,23 @@ int veda_tile_scores_noalloc(const veda_layer* L, const float* dq, const float* 
 int veda_topk_mask(const veda_layer* L, const float* scores, const int32_t* k, int32_t k_cap,
                    int32_t* idx, uint8_t* mask, cudaStream_t stream);
 
+/* Tile scores and the top-k mask in one call (Veda summary 2.1; the pages
+ * name tighter kernel fusion as future work): the per-head MLP of
+ * veda_tile_scores into emb_ws, then one kernel that builds whole score rows
+ * in shared memory and selects from them, so the score matrix need not go
+ * through HBM. Arguments as in veda_tile_scores and veda_topk_mask; `scores`
+ * may be NULL (then it is not written) or receive the same matrix
+ * veda_tile_scores writes. idx, mask and scores are bit-identical to
+ * veda_tile_scores followed by veda_topk_mask. A score row must fit shared
+ * memory (4*nt_cap + 4*out_dim + 8192 <= 204800 bytes, true for every layer
+ * the library accepts), else VEDA_ERR_UNSUPPORTED. Measured slower than the
+ * two separate calls on the 153,600-token layer (1.07 vs 0.85 ms). */
+int veda_tile_scores_topk(const veda_layer* L, const float* dq, const float* dk,
+                          const float* w1q, const float* b1q, const float* w2q, const float* b2q,
+                          const float* w1k, const float* b1k, const float* w2k, const float* b2k,
+                          int32_t hidden, int32_t out_dim, float scale, const int32_t* k, int32_t k_cap,
+                          int32_t* idx, uint8_t* mask, float* scores, float* emb_ws, cudaStream_t stream);
+
 /* Tile-skipping sparse attention (Veda summary 2.3): for each query row i of
  * query tile a, O_i = sum_j softmax_j(scale * q_i . k_j) v_j over the valid
  * keys j of the key tiles idx[a, 0..k[h]) only; the softmax is renormalised

@@ -170,6 +170,62 @@ def test_tile_scores(name):
             assert not got[b, h, nt:].any() and not got[b, h, :, nt:].any()
 
 
+def _scores_topk_pair(w, zero_out=False, seed=5):
+    """Unfused (scores, then top-k) and fused outputs on the same random
+    descriptors and weights."""
+    L = _layer(w)
+    nt_cap = L.nt_cap
+    rng = np.random.default_rng(seed)
+    dq = rng.standard_normal((w.B, w.heads, nt_cap, 3 * w.d)).astype(np.float32)
+    dk = rng.standard_normal((w.B, w.heads, nt_cap, 3 * w.d)).astype(np.float32)
+    w1, b1, w2, b2 = synth.mlp_weights(w)
+    b1 = rng.standard_normal(b1.shape).astype(np.float32) * 0.1
+    b2 = rng.standard_normal(b2.shape).astype(np.float32) * 0.1
+    if zero_out:                       # every score 0: the tie rule alone decides
+        w2, b2 = np.zeros_like(w2), np.zeros_like(b2)
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    args = [T(a) for a in (dq, dk, w1, b1, w2, b2, w1, b1, w2, b2)]
+    ks = [max(1, (L.nt[h] * (h + 1)) // (3 * w.heads)) for h in range(w.heads)]
+    k_cap = max(ks) + 2
+    ws = torch.empty(V.veda_tile_scores_ws_bytes(L, 64) // 4, dtype=torch.float32, device=DEV)
+    s1 = torch.empty((w.B, w.heads, nt_cap, nt_cap), dtype=torch.float32, device=DEV)
+    i1 = torch.empty((w.B, w.heads, nt_cap, k_cap), dtype=torch.int32, device=DEV)
+    m1 = torch.empty((w.B, w.heads, nt_cap, nt_cap), dtype=torch.uint8, device=DEV)
+    V.veda_tile_scores(L, *args, 128, 64, synth.SCORE_SCALE, s1, ws)
+    V.veda_topk_mask(L, s1, ks, k_cap, i1, m1)
+    s2, i2, m2 = torch.full_like(s1, 7.0), torch.full_like(i1, 7), torch.full_like(m1, 7)
+    V.veda_tile_scores_topk(L, *args, 128, 64, synth.SCORE_SCALE, ks, k_cap, i2, ws, mask=m2, scores=s2)
+    i3 = torch.full_like(i1, 7)
+    V.veda_tile_scores_topk(L, *args, 128, 64, synth.SCORE_SCALE, ks, k_cap, i3, ws)
+    V.veda_check_status(L)
+    return L, ks, k_cap, (s1, i1, m1), (s2, i2, m2), i3
+
+
+@pytest.mark.parametrize("name", list(WL))
+@pytest.mark.parametrize("zero_out", [False, True])
+def test_tile_scores_topk_fused(name, zero_out):
+    """The fused call gives bit-identical scores, index lists and mask to the
+    two unfused calls (with and without the optional outputs), and its lists
+    are the oracle's top-k of those scores."""
+    w = WL[name]
+    L, ks, k_cap, (s1, i1, m1), (s2, i2, m2), i3 = _scores_topk_pair(w, zero_out)
+    assert torch.equal(s1, s2) and torch.equal(i1, i2) and torch.equal(m1, m2) and torch.equal(i1, i3)
+    sc, gi = s1.cpu().numpy(), i2.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt = L.nt[h]
+            ri, _ = O.topk_rows(sc[b, h, :nt, :nt], ks[h], k_cap)
+            assert np.array_equal(gi[b, h, :nt], ri)
+            assert (gi[b, h, nt:] == -1).all()
+
+
+def test_tile_scores_topk_fused_long_rows():
+    """8,000 key tiles per row: fewer rows per CTA (6) fit shared memory."""
+    w = synth.custom("long", 1, 2, 64, 8000, 8, 8, 64, [(1, 8, 8), (1, 8, 8)], 0.1, 31)
+    L, ks, k_cap, (s1, i1, m1), (s2, i2, m2), i3 = _scores_topk_pair(w)
+    assert torch.equal(s1, s2) and torch.equal(i1, i2) and torch.equal(m1, m2) and torch.equal(i1, i3)
+
+
 # -------------------------------------------------------------------- top-k
 
 def _topk_case(w, scores_np, k):
