@@ -30,6 +30,7 @@ __all__ = [
     "head_layout", "perm_indices", "permute", "unpermute", "trippool", "gelu",
     "mlp", "tile_scores", "topk_rows", "sparse_attention", "full_tilemap",
     "kl_rows", "recall", "k_from_keep", "effective_pairs",
+    "gelu_grad", "estimator_loss", "estimator_grad",
 ]
 
 
@@ -271,3 +272,65 @@ def effective_pairs(lens, idx_h, k, rows=None):
     kl = np.asarray(lens, np.int64)
     return int(sum(int(kl[a]) * int(kl[np.asarray(idx_h[a, :k])].sum()) for a in rows))
 
+
+
+# ---------------------------------------------------------------------------
+# 8. estimator training (Veda summary 2.1, "Optimization": the head-specific
+#    projections are trained with a row-wise KL against the oracle tile map,
+#    with stop-gradient on the pooled descriptors; 2.3, "Training Efficiency":
+#    on random subsets of query tiles)
+# ---------------------------------------------------------------------------
+
+def gelu_grad(x):
+    """d/dx of the exact GELU: Phi(x) + x * phi(x), phi the standard normal
+    density."""
+    x = np.asarray(x, np.float64)
+    erf = np.vectorize(math.erf, otypes=[np.float64])
+    return 0.5 * (1.0 + erf(x / math.sqrt(2.0))) + x * np.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+
+
+def estimator_loss(dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scale, M_rows):
+    """[reading] One head's distillation loss: the mean over the sampled query
+    tiles (rows of dq_rows, with their tile-map rows M_rows) of KL(t || p),
+    t = map row / its sum, p = softmax of the predicted score row over all of
+    the head's key tiles (dk). Scores stay fp64 here (no fp32 rounding), so
+    the loss is a smooth function of the weights."""
+    q = mlp(dq_rows, w1q, b1q, w2q, b2q)
+    k = mlp(dk, w1k, b1k, w2k, b2k)
+    return float(kl_rows(M_rows, q @ k.T * scale).mean())
+
+
+def estimator_grad(dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scale, M_rows):
+    """Gradient of estimator_loss with respect to the eight weight arrays,
+    returned as a dict {"w1q", "b1q", "w2q", "b2q", "w1k", ...} in the
+    weights' own shapes; descriptors and the tile map are constants.
+
+    Chain rule, written out: with G = (p - t) / rows the gradient of the loss
+    with respect to the score matrix (KL(t || softmax(s)) has gradient p - t
+    in s because t sums to 1), the score s = scale * q k^T gives
+    dq = scale G k and dk = scale G^T q; each side's MLP y = GELU(x W1 + b1)
+    W2 + b2 then gives dW2 = GELU(z)^T dy, db2 = sum dy, dz = (dy W2^T) *
+    GELU'(z), dW1 = x^T dz, db1 = sum dz."""
+    f = lambda a: np.asarray(a, np.float64)
+    xq, xk = f(dq_rows), f(dk)
+    zq = xq @ f(w1q) + f(b1q)
+    zk = xk @ f(w1k) + f(b1k)
+    hq, hk = gelu(zq), gelu(zk)
+    q = hq @ f(w2q) + f(b2q)
+    k = hk @ f(w2k) + f(b2k)
+    s = q @ k.T * scale
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    M = f(M_rows)
+    t = M / M.sum(axis=1, keepdims=True)
+    G = (p - t) / s.shape[0]
+    dy = {"q": scale * G @ k, "k": scale * G.T @ q}
+    out = {}
+    for side, x, z, h, w2 in (("q", xq, zq, hq, f(w2q)), ("k", xk, zk, hk, f(w2k))):
+        g = dy[side]
+        dz = (g @ w2.T) * gelu_grad(z)
+        out["w1" + side] = x.T @ dz
+        out["b1" + side] = dz.sum(axis=0)
+        out["w2" + side] = h.T @ g
+        out["b2" + side] = g.sum(axis=0)
+    return out

@@ -349,3 +349,75 @@ def test_recall_and_effective_pairs():
     lens = np.array([4, 4, 2])
     idx = np.array([[0, 2], [1, 2], [0, 1]])
     assert O.effective_pairs(lens, idx, 2) == 4 * 6 + 4 * 6 + 2 * 8
+
+
+# ------------------------------------------------- estimator training (gradients)
+
+_WNAMES = ["w1q", "b1q", "w2q", "b2q", "w1k", "b1k", "w2k", "b2k"]
+
+
+def _estimator_problem(seed=0, d3=6, hid=5, od=4, nt=7, nr=3):
+    rng = np.random.default_rng(seed)
+    W = {"w1q": rng.standard_normal((d3, hid)), "b1q": rng.standard_normal(hid) * 0.1,
+         "w2q": rng.standard_normal((hid, od)), "b2q": rng.standard_normal(od) * 0.1,
+         "w1k": rng.standard_normal((d3, hid)), "b1k": rng.standard_normal(hid) * 0.1,
+         "w2k": rng.standard_normal((hid, od)), "b2k": rng.standard_normal(od) * 0.1}
+    dq = rng.standard_normal((nr, d3))
+    dk = rng.standard_normal((nt, d3))
+    M = rng.uniform(0.01, 1.0, (nr, nt))
+    M[0, 2] = 0.0                                   # a zero map entry (0 log 0 = 0)
+    return W, dq, dk, M
+
+
+def test_estimator_grad_finite_differences():
+    """Every entry of every weight gradient against a central difference of
+    the loss (fp64, step 1e-5): pins each term of the chain rule."""
+    W, dq, dk, M = _estimator_problem()
+    scale = 0.3
+    loss = lambda: O.estimator_loss(dq, dk, *[W[n] for n in _WNAMES], scale, M)
+    g = O.estimator_grad(dq, dk, *[W[n] for n in _WNAMES], scale, M)
+    for n in _WNAMES:
+        a = W[n]
+        assert g[n].shape == a.shape
+        fd = np.zeros_like(a)
+        for i in np.ndindex(a.shape):
+            old = a[i]
+            a[i] = old + 1e-5
+            lp = loss()
+            a[i] = old - 1e-5
+            lm = loss()
+            a[i] = old
+            fd[i] = (lp - lm) / 2e-5
+        np.testing.assert_allclose(g[n], fd, rtol=0, atol=1e-8 * max(1.0, np.abs(fd).max()), err_msg=n)
+
+
+def test_estimator_grad_invariants_and_autograd():
+    W, dq, dk, M = _estimator_problem(seed=1)
+    args = [W[n] for n in _WNAMES]
+    g = O.estimator_grad(dq, dk, *args, 0.3, M)
+    # a shift of every key embedding adds a per-row constant to the scores:
+    # softmax, and so the loss, cannot depend on the key-side output bias
+    np.testing.assert_allclose(g["b2k"], 0.0, atol=1e-14)
+    # at the minimum (target = the predicted distribution) every gradient is 0
+    q = O.mlp(dq, *args[:4])
+    k = O.mlp(dk, *args[4:])
+    s = q @ k.T * 0.3
+    p = np.exp(s - s.max(1, keepdims=True))
+    g0 = O.estimator_grad(dq, dk, *args, 0.3, 5.0 * p / p.sum(1, keepdims=True))
+    for n in _WNAMES:
+        np.testing.assert_allclose(g0[n], 0.0, atol=1e-13)
+    # GELU derivative: value at 0, and a difference quotient elsewhere
+    assert O.gelu_grad(0.0) == pytest.approx(0.5, abs=1e-15)
+    x = np.linspace(-4, 4, 17)
+    np.testing.assert_allclose(O.gelu_grad(x), (O.gelu(x + 1e-6) - O.gelu(x - 1e-6)) / 2e-6, atol=1e-8)
+    # torch autograd (fp64) on the same loss, built from torch's own ops
+    T = {n: torch.tensor(W[n], dtype=torch.float64, requires_grad=True) for n in _WNAMES}
+    gel = torch.nn.functional.gelu
+    xq, xk = torch.from_numpy(dq), torch.from_numpy(dk)
+    qt = gel(xq @ T["w1q"] + T["b1q"]) @ T["w2q"] + T["b2q"]
+    kt = gel(xk @ T["w1k"] + T["b1k"]) @ T["w2k"] + T["b2k"]
+    lp = torch.log_softmax(qt @ kt.T * 0.3, dim=1)
+    tt = torch.from_numpy(M / M.sum(1, keepdims=True))
+    torch.nn.functional.kl_div(lp, tt, reduction="none").sum(1).mean().backward()
+    for n in _WNAMES:
+        np.testing.assert_allclose(g[n], T[n].grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=n)

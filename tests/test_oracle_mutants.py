@@ -96,6 +96,23 @@ def _gelu_tanh(x):
     return 0.5 * x * (1 + np.tanh(math.sqrt(2 / math.pi) * (x + 0.044715 * x ** 3)))
 
 
+def _grad_no_row_mean(dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scale, M_rows):
+    """slip: gradient of the row sum instead of the row mean."""
+    g = _orig["estimator_grad"](dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scale, M_rows)
+    return {n: v * np.asarray(dq_rows).shape[0] for n, v in g.items()}
+
+
+def _gelu_grad_as_gelu(x):
+    """slip: GELU itself used where its derivative belongs."""
+    return _orig["gelu"](x)
+
+
+def _grad_sign_flipped(dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scale, M_rows):
+    """slip: t - p instead of p - t (ascent direction)."""
+    g = _orig["estimator_grad"](dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scale, M_rows)
+    return {n: -v for n, v in g.items()}
+
+
 CASES = [
     ("perm_indices", _perm_x_major, ["test_perm_golden"]),
     ("trippool", _trippool_no_max, ["test_trippool_golden", "test_trippool_invariants_and_brute_force"]),
@@ -106,6 +123,10 @@ CASES = [
     ("full_tilemap", _tilemap_mean, ["test_tilemap_brute_force", "test_tilemap_one_hot_gives_expected_mask"]),
     ("kl_rows", _kl_reversed, ["test_kl_golden_and_invariants"]),
     ("gelu", _gelu_tanh, ["test_gelu_golden", "test_mlp_against_loops"]),
+    ("estimator_grad", _grad_no_row_mean, ["test_estimator_grad_finite_differences"]),
+    ("gelu_grad", _gelu_grad_as_gelu, ["test_estimator_grad_finite_differences"]),
+    ("estimator_grad", _grad_sign_flipped, ["test_estimator_grad_finite_differences",
+                                            "test_estimator_grad_invariants_and_autograd"]),
 ]
 
 
