@@ -28,7 +28,7 @@ VEDA_ERR_BAD_INDEX = -5
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
             "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
-            "veda_selftest_wait_timeout", "veda_last_error")
+            "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_selftest_wait_timeout", "veda_last_error")
 
 
 class VedaError(RuntimeError):
@@ -72,12 +72,15 @@ _lib.veda_topk_mask.argtypes = [_LP, _P, _P, _I, _P, _P, _P]
 _lib.veda_tile_scores_topk.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _P, _P, _P, _P]
 _lib.veda_sparse_attn.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
 _lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P, _P, _P, _P, _P]
+_lib.veda_estimator_grad.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _I, _P] + [_P] * 8 + [_P, _P, _P]
+_lib.veda_estimator_grad_ws_bytes.argtypes = [_LP, _I, _I, _I, _I]
+_lib.veda_estimator_grad_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_check_status.argtypes = [_LP, _P]
 _lib.veda_selftest_wait_timeout.argtypes = [_LP, ctypes.c_uint32, _P]
 _lib.veda_last_error.restype = ctypes.c_char_p
 for _name in EXPORTED:
     getattr(_lib, _name)
-    if _name not in ("veda_last_error", "veda_tile_scores_ws_bytes"):
+    if _name not in ("veda_last_error", "veda_tile_scores_ws_bytes", "veda_estimator_grad_ws_bytes"):
         getattr(_lib, _name).restype = ctypes.c_int
 
 
@@ -208,6 +211,21 @@ def veda_full_attn_tilemax(layer: Layer, qp, kp, heads_sel: Sequence[int], qtile
     _check(_lib.veda_full_attn_tilemax(layer.ref, _ptr(qp), _ptr(kp), _host_i32(heads_sel), len(heads_sel),
                                        _ptr(qtile_rows), int(n_rows), float(scale), _ptr(tilemap), _ptr(lse),
                                        _ptr(scores), _ptr(kl_rows), _ptr(kl_out), _stream(stream)))
+
+
+def veda_estimator_grad_ws_bytes(layer: Layer, n_heads_sel: int, n_rows: int, hidden: int, out_dim: int) -> int:
+    return int(_lib.veda_estimator_grad_ws_bytes(layer.ref, n_heads_sel, n_rows, hidden, out_dim))
+
+
+def veda_estimator_grad(layer: Layer, dq, dk, weights: Sequence[torch.Tensor], hidden: int, out_dim: int,
+                        scale: float, heads_sel: Sequence[int], qtile_rows: Optional[torch.Tensor], n_rows: int,
+                        tilemap: torch.Tensor, grads: Sequence[torch.Tensor], ws: torch.Tensor,
+                        loss: Optional[torch.Tensor] = None, stream=None):
+    """weights and grads: (w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k)."""
+    _check(_lib.veda_estimator_grad(layer.ref, _ptr(dq), _ptr(dk), *[_ptr(t) for t in weights], hidden, out_dim,
+                                    float(scale), _host_i32(heads_sel), len(heads_sel), _ptr(qtile_rows),
+                                    int(n_rows), _ptr(tilemap), *[_ptr(t) for t in grads], _ptr(loss), _ptr(ws),
+                                    _stream(stream)))
 
 
 def veda_check_status(layer: Layer, stream=None):

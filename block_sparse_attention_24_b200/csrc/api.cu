@@ -309,6 +309,59 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp, 
                       "veda_full_attn_tilemax");
 }
 
+size_t veda_estimator_grad_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows, int32_t hidden,
+                                    int32_t out_dim) {
+  veda::LayerGeom g;
+  if (build_geom(L, &g) != VEDA_OK || n_heads_sel < 1 || n_rows < 1 || hidden < 1 || out_dim < 1) return 0;
+  return (size_t)n_heads_sel * veda::estimator_ws_floats_per_head(g.nt_cap, n_rows, hidden, out_dim) * sizeof(float);
+}
+
+int veda_estimator_grad(const veda_layer* L, const float* dq, const float* dk, const float* w1q, const float* b1q,
+                        const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
+                        const float* b2k, int32_t hidden, int32_t out_dim, float scale, const int32_t* heads_sel,
+                        int32_t n_heads_sel, const int32_t* qtile_rows, int32_t n_rows, const float* tilemap,
+                        float* g_w1q, float* g_b1q, float* g_w2q, float* g_b2q, float* g_w1k, float* g_b1k,
+                        float* g_w2k, float* g_b2k, float* loss, float* ws, cudaStream_t stream) {
+  veda::LayerGeom g;
+  VEDA_TRY(build_geom(L, &g));
+  if (g.B != 1) return fail(VEDA_ERR_UNSUPPORTED, "estimator gradient: only B == 1 layers are accepted");
+  const float* w[8] = {w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k};
+  float* gw[8] = {g_w1q, g_b1q, g_w2q, g_b2q, g_w1k, g_b1k, g_w2k, g_b2k};
+  const char* wn[8] = {"w1q", "b1q", "w2q", "b2q", "w1k", "b1k", "w2k", "b2k"};
+  const char* gn[8] = {"g_w1q", "g_b1q", "g_w2q", "g_b2q", "g_w1k", "g_b1k", "g_w2k", "g_b2k"};
+  VEDA_TRY(check_ptr(dq, "dq"));
+  VEDA_TRY(check_ptr(dk, "dk"));
+  for (int i = 0; i < 8; ++i) {
+    VEDA_TRY(check_ptr(w[i], wn[i]));
+    VEDA_TRY(check_ptr(gw[i], gn[i]));
+  }
+  VEDA_TRY(check_ptr(tilemap, "tilemap"));
+  VEDA_TRY(check_ptr(ws, "ws"));
+  if (qtile_rows) VEDA_TRY(check_ptr(qtile_rows, "qtile_rows"));
+  if (loss) VEDA_TRY(check_ptr(loss, "loss"));
+  if (hidden < 4 || hidden > 256 || hidden % 4)
+    return fail(VEDA_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 4 in [4, 256]", hidden);
+  if (out_dim < 4 || out_dim > 128 || out_dim % 4)
+    return fail(VEDA_ERR_UNSUPPORTED, "out_dim=%d must be a multiple of 4 in [4, 128]", out_dim);
+  if (!heads_sel || n_heads_sel < 1 || n_heads_sel > VEDA_MAX_HEADS)
+    return fail(VEDA_ERR_INVALID_ARG, "heads_sel must list 1..%d heads", VEDA_MAX_HEADS);
+  if (n_rows < 1 || n_rows > g.nt_cap) return fail(VEDA_ERR_INVALID_ARG, "n_rows=%d outside [1, nt_cap]", n_rows);
+  if (!(scale > 0.f) || scale != scale || scale > 3.0e38f)
+    return fail(VEDA_ERR_INVALID_ARG, "scale must be positive and finite");
+  for (int s = 0; s < n_heads_sel; ++s) {
+    if (heads_sel[s] < 0 || heads_sel[s] >= g.heads)
+      return fail(VEDA_ERR_INVALID_ARG, "heads_sel[%d]=%d outside [0, %d)", s, heads_sel[s], g.heads);
+    for (int t = 0; t < s; ++t)
+      if (heads_sel[t] == heads_sel[s]) return fail(VEDA_ERR_INVALID_ARG, "heads_sel lists head %d twice", heads_sel[s]);
+    if (!qtile_rows && n_rows > g.h[heads_sel[s]].nt)
+      return fail(VEDA_ERR_INVALID_ARG, "n_rows=%d exceeds the %d tiles of head %d", n_rows,
+                  g.h[heads_sel[s]].nt, heads_sel[s]);
+  }
+  return after_launch(veda::launch_estimator_grad(g, dq, dk, w, gw, hidden, out_dim, scale, heads_sel, n_heads_sel,
+                                                  qtile_rows, n_rows, tilemap, loss, ws, stream),
+                      "veda_estimator_grad");
+}
+
 int veda_check_status(const veda_layer* L, cudaStream_t stream) {
   if (!L || !L->dev_status) return fail(VEDA_ERR_INVALID_ARG, "layer or dev_status is NULL");
   cudaError_t e = cudaStreamSynchronize(stream);

@@ -196,6 +196,36 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp,
                            float* tilemap, float* lse, const float* scores,
                            float* kl_rows, float* kl_out, cudaStream_t stream);
 
+/* Estimator training (Veda summary 2.1, Optimization: the head-specific
+ * projections are trained with the row-wise KL against the tile map, with
+ * stop-gradient on the pooled descriptors; 2.3, Training Efficiency: on
+ * random subsets of query tiles). For the selected heads heads_sel (HOST,
+ * distinct) and their sampled query tiles qtile_rows [n_heads_sel, n_rows]
+ * (DEVICE; NULL = tiles 0..n_rows-1), with tilemap the output of
+ * veda_full_attn_tilemax for the same heads and rows, computes
+ *   loss = mean over heads of mean over rows of KL(t || softmax(s_row)),
+ *   s_row[j] = scale * MLP_q(dq[row]) . MLP_k(dk[j]) over the head's tiles,
+ * and writes its gradient with respect to every weight array into g_* (same
+ * shapes as the weights: g_w1q [heads,3d,hidden], g_b1q [heads,hidden],
+ * g_w2q [heads,hidden,out_dim], g_b2q [heads,out_dim], and the key side);
+ * heads not selected get zeros. Query and key weights get separate
+ * gradients (sum them when one MLP serves both). *loss (device fp32, may be
+ * NULL) receives the loss. Scores are recomputed in fp32 from the weights
+ * given. ws: veda_estimator_grad_ws_bytes(...) bytes of device scratch.
+ * fp32 arithmetic; every reduction in a fixed order (bit-reproducible).
+ * Only B == 1 layers are accepted. */
+size_t veda_estimator_grad_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows,
+                                    int32_t hidden, int32_t out_dim);
+int veda_estimator_grad(const veda_layer* L, const float* dq, const float* dk,
+                        const float* w1q, const float* b1q, const float* w2q, const float* b2q,
+                        const float* w1k, const float* b1k, const float* w2k, const float* b2k,
+                        int32_t hidden, int32_t out_dim, float scale,
+                        const int32_t* heads_sel, int32_t n_heads_sel,
+                        const int32_t* qtile_rows, int32_t n_rows, const float* tilemap,
+                        float* g_w1q, float* g_b1q, float* g_w2q, float* g_b2q,
+                        float* g_w1k, float* g_b1k, float* g_w2k, float* g_b2k,
+                        float* loss, float* ws, cudaStream_t stream);
+
 /* Diagnostic (no counterpart on the pages): launches one thread that waits,
  * through the bounded wait every pipeline kernel uses, on a barrier nothing
  * arrives on. After limit_ms (1..10000) the wait gives up and records
