@@ -233,6 +233,7 @@ def run_ours(args, world, rank, local):
 
     # per-stage breakdown of the front end (separate, untimed-for-value pass)
     stage_ms = stage_breakdown(V, L, layer, q, k, v, stream)
+    grad_ms = estimator_grad_ms(layer, stream)
 
     # dense path (same kernel, every tile kept) on the same permuted tensors
     dense_out = torch.empty_like(layer.op)
@@ -275,6 +276,7 @@ def run_ours(args, world, rank, local):
         "layer_ms": round(front_ms + attn_ms + unperm_ms, 3),
         "stage_ms": {**stage_ms, "front_end": round(front_ms, 3), "sparse_attn": round(attn_ms, 3),
                      "unpermute": round(unperm_ms, 3), "tilemap_kl": round(map_ms, 3)},
+        "estimator_grad_ms": grad_ms,
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": sustained, "unit": UNIT,
                      "frac": round(attn_tflops / sustained, 4), "traffic": traffic,
                      "kernel": "sparse_attn_pair_kernel<128>",
@@ -310,6 +312,21 @@ def stage_breakdown(V, L, layer, q, k, v, stream):
     ev[4].record(stream)
     torch.cuda.synchronize()
     return {n: round(ev[i].elapsed_time(ev[i + 1]), 3) for i, n in enumerate(names)}
+
+
+def estimator_grad_ms(layer, stream, reps=5):
+    """One estimator-training gradient (the KL back through the score product
+    and the MLP, on this step's tile-map rows): outside the step, reported
+    beside it."""
+    layer.estimator_grad()
+    layer.estimator_grad()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        layer.estimator_grad()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return round(e0.elapsed_time(e1) / reps, 3)
 
 
 def run_e2e(V, L, layer, q, k, v, device, eff_flops, args):

@@ -17,8 +17,8 @@ from typing import Dict, List, Optional, Sequence
 
 import torch
 
-from . import (Layer, veda_full_attn_tilemax, veda_permute, veda_permute_trippool, veda_sparse_attn,
-               veda_tile_scores, veda_tile_scores_ws_bytes, veda_topk_mask)
+from . import (Layer, veda_estimator_grad, veda_estimator_grad_ws_bytes, veda_full_attn_tilemax, veda_permute,
+               veda_permute_trippool, veda_sparse_attn, veda_tile_scores, veda_tile_scores_ws_bytes, veda_topk_mask)
 
 
 def k_from_keep(keep: float, nt: int) -> int:
@@ -115,6 +115,26 @@ class VedaLayer:
         m = self.maps
         veda_full_attn_tilemax(self.L, self.qp, self.kp, m.heads, m.rows, m.n_rows, self.attn_scale, self.tilemap,
                                self.map_lse, self.scores, self.kl_rows, self.kl_out, stream=stream)
+
+    def estimator_grad(self, stream=None):
+        """Weight gradient of the distillation loss on this step's tile-map
+        rows (call after distill()): returns the eight gradient arrays
+        (w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k) and the loss, on the device.
+        The layer ties one MLP to both sides, so its gradient is the sum of
+        the query and key parts."""
+        m = self.maps
+        if m is None:
+            raise ValueError("estimator_grad needs tile-map rows (maps=...)")
+        names = ("w1q", "b1q", "w2q", "b2q", "w1k", "b1k", "w2k", "b2k")
+        if not hasattr(self, "_grads"):
+            self._grads = [torch.empty_like(self.w[n]) for n in names]
+            self._grad_loss = torch.empty(1, dtype=torch.float32, device=self.device)
+            nbytes = veda_estimator_grad_ws_bytes(self.L, len(m.heads), m.n_rows, self.hidden, self.out_dim)
+            self._grad_ws = torch.empty(nbytes // 4, dtype=torch.float32, device=self.device)
+        veda_estimator_grad(self.L, self.dq, self.dk, [self.w[n] for n in names], self.hidden, self.out_dim,
+                            self.score_scale, m.heads, m.rows, m.n_rows, self.tilemap, self._grads, self._grad_ws,
+                            self._grad_loss, stream=stream)
+        return self._grads, self._grad_loss
 
     def forward(self, q, k, v, stream=None):
         self.front(q, k, v, stream)

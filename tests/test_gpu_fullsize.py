@@ -146,3 +146,35 @@ def test_dense_path_full_size_sampled():
         op = _f64(out[0, h])
         e = np.concatenate([np.abs(op[a * w.tile: a * w.tile + lens[a]] - oa).ravel() for a, (oa, _) in ref.items()])
         assert e.max() <= 2e-2 and e.mean() <= 2e-3, (e.max(), e.mean())
+
+
+def test_estimator_grad_full_size():
+    """The weight gradient of the distillation loss at the 153,600-token
+    layer (2 heads x 120 sampled query tiles over 1,200 key tiles) against the
+    fp64 oracle, from the layer's own descriptors and tile map."""
+    w = synth.config(3)
+    V, L, layer, (q, k, v) = bench.build_layer(w, DEV)
+    layer.forward(q, k, v)
+    grads, loss = layer.estimator_grad()
+    V.veda_check_status(L)
+    m = layer.maps
+    rows = m.rows.cpu().numpy()
+    xq, xk = _f64(layer.dq[0]), _f64(layer.dk[0])
+    M = layer.tilemap.cpu().double().numpy()
+    np_w = synth.mlp_weights(w)
+    names = ["w1q", "b1q", "w2q", "b2q", "w1k", "b1k", "w2k", "b2k"]
+    got = [g.cpu().double().numpy() for g in grads]
+    losses = []
+    for s, h in enumerate(m.heads):
+        nt = L.nt[h]
+        args = [a[h].astype(np.float64) for a in np_w] * 2
+        g = O.estimator_grad(xq[h, rows[s]], xk[h, :nt], *args, synth.SCORE_SCALE, M[s, :, :nt])
+        losses.append(O.estimator_loss(xq[h, rows[s]], xk[h, :nt], *args, synth.SCORE_SCALE, M[s, :, :nt]))
+        for side in (0, 1):
+            scale = max(np.abs(g[n]).max() for n in names[4 * side: 4 * side + 4]) / len(m.heads)
+            for i in range(4 * side, 4 * side + 4):
+                err = np.abs(got[i][h] - g[names[i]] / len(m.heads)).max()
+                assert err <= 2e-3 * scale, (names[i], h, err, scale)
+    for h in set(range(w.heads)) - set(m.heads):
+        assert not any(got[i][h].any() for i in range(8))
+    assert float(loss.item()) == pytest.approx(float(np.mean(losses)), rel=1e-4)
