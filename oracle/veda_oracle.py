@@ -30,7 +30,7 @@ __all__ = [
     "head_layout", "perm_indices", "permute", "unpermute", "trippool", "gelu",
     "mlp", "tile_scores", "topk_rows", "sparse_attention", "full_tilemap",
     "kl_rows", "recall", "k_from_keep", "effective_pairs",
-    "gelu_grad", "estimator_loss", "estimator_grad",
+    "gelu_grad", "estimator_loss", "estimator_grad", "tiling_errors",
 ]
 
 
@@ -334,3 +334,46 @@ def estimator_grad(dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scale, M
         out["w2" + side] = h.T @ g
         out["b2" + side] = g.sum(axis=0)
     return out
+
+
+# ---------------------------------------------------------------------------
+# 9. head-aware tiling search (Veda summary 2.2: a tiling per head, chosen
+#    offline on calibration inputs to match that head's locality)
+# ---------------------------------------------------------------------------
+
+def tiling_errors(q, k, v, T, H, W, candidates, keep, scale):
+    """[reading] Calibration score of each candidate tiling for each head:
+    squared Frobenius distance, over the head's tokens, between full attention
+    and the tile-skipping attention that keeps, for every query tile, the k
+    key tiles with the largest oracle tile-map values (the mask the estimator
+    is distilled towards), all under that tiling. The chosen tiling of head h
+    is argmin over candidates of errors[c, h].
+
+    q, k, v: [1, N, heads, d] (bf16 values). Returns errors [len(candidates),
+    heads] (fp64)."""
+    q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+    B, N, Hh, d = q.shape
+    assert B == 1
+    # full attention in the original order, per head (tiling-independent)
+    full = np.zeros((N, Hh, d))
+    for h in range(Hh):
+        s = q[0, :, h] @ k[0, :, h].T * scale
+        w = np.exp(s - s.max(axis=1, keepdims=True))
+        full[:, h] = (w / w.sum(axis=1, keepdims=True)) @ v[0, :, h]
+    errors = np.zeros((len(candidates), Hh))
+    for c, tiling in enumerate(candidates):
+        lay = head_layout(T, H, W, tiling)
+        perm = perm_indices(T, H, W, tiling)
+        perms = [perm] * Hh
+        nt, lens, tile = lay["nt"], lay["lens"], lay["tile"]
+        kk = k_from_keep(keep, nt)
+        qp, kp, vp = (permute(a, perms, lay["n_pad"]) for a in (q, k, v))
+        op = np.zeros((1, Hh, lay["n_pad"], d))
+        for h in range(Hh):
+            M, _ = full_tilemap(qp[0, h], kp[0, h], lens, tile, scale)
+            idx, _ = topk_rows(M.astype(np.float32), kk)
+            for a, (oa, _) in sparse_attention(qp[0, h], kp[0, h], vp[0, h], idx, kk, lens, tile, scale).items():
+                op[0, h, a * tile: a * tile + int(lens[a])] = oa
+        o = unpermute(op, perms, N)[0]
+        errors[c] = ((o - full) ** 2).sum(axis=(0, 2))
+    return errors

@@ -421,3 +421,33 @@ def test_estimator_grad_invariants_and_autograd():
     torch.nn.functional.kl_div(lp, tt, reduction="none").sum(1).mean().backward()
     for n in _WNAMES:
         np.testing.assert_allclose(g[n], T[n].grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=n)
+
+
+# ------------------------------------------------------ head-aware tiling search
+
+def test_tiling_errors_keep_all_and_designed_locality():
+    """keep = 1 keeps every tile, so every candidate reproduces full attention
+    (error 0). With attention confined to each token's own frame (one t), a
+    tiling whose tiles are whole frames keeps exactly the right key tile at
+    k = 1 (error ~ 0) while tilings that mix frames cannot; head 1 is built
+    local in x-columns instead (every frame at one x), which tiles spanning
+    all of T (one x column each) capture."""
+    T, H, W, d = 4, 2, 4, 8
+    N = T * H * W
+    t, y, x = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    t, y, x = t.ravel(), y.ravel(), x.ravel()
+    q = np.zeros((1, N, 2, d))
+    k = np.zeros((1, N, 2, d))
+    beta = 12.0
+    q[0, np.arange(N), 0, t] = beta                 # head 0: one-hot of the frame
+    k[0, np.arange(N), 0, t] = beta
+    q[0, np.arange(N), 1, x] = beta                 # head 1: one-hot of the x column
+    k[0, np.arange(N), 1, x] = beta
+    v = np.random.default_rng(3).standard_normal((1, N, 2, d))
+    cands = [(1, 2, 4), (4, 2, 1)]                  # whole frames | whole x columns over time
+    e_all = O.tiling_errors(q, k, v, T, H, W, cands, 1.0, 1.0)
+    np.testing.assert_allclose(e_all, 0.0, atol=1e-20)
+    e = O.tiling_errors(q, k, v, T, H, W, cands, 0.25, 1.0)   # k = 1 of 4 tiles
+    assert e[0, 0] < 1e-20 and e[1, 0] > 1e-3                # head 0 wants frames
+    assert e[1, 1] < 1e-20 and e[0, 1] > 1e-3                # head 1 wants x columns
+    assert list(np.argmin(e, axis=0)) == [0, 1]

@@ -113,6 +113,11 @@ def _grad_sign_flipped(dq_rows, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scal
     return {n: -v for n, v in g.items()}
 
 
+def _tiling_errors_sparsity_for_keep(q, k, v, T, H, W, candidates, keep, scale):
+    """slip: the sparsity (1 - keep) used where the keep fraction belongs."""
+    return _orig["tiling_errors"](q, k, v, T, H, W, candidates, 1.0 - keep, scale)
+
+
 CASES = [
     ("perm_indices", _perm_x_major, ["test_perm_golden"]),
     ("trippool", _trippool_no_max, ["test_trippool_golden", "test_trippool_invariants_and_brute_force"]),
@@ -127,6 +132,7 @@ CASES = [
     ("gelu_grad", _gelu_grad_as_gelu, ["test_estimator_grad_finite_differences"]),
     ("estimator_grad", _grad_sign_flipped, ["test_estimator_grad_finite_differences",
                                             "test_estimator_grad_invariants_and_autograd"]),
+    ("tiling_errors", _tiling_errors_sparsity_for_keep, ["test_tiling_errors_keep_all_and_designed_locality"]),
 ]
 
 
