@@ -28,7 +28,7 @@ VEDA_ERR_BAD_INDEX = -5
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
             "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
-            "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_selftest_wait_timeout", "veda_last_error")
+            "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_output_sq_error", "veda_selftest_wait_timeout", "veda_last_error")
 
 
 class VedaError(RuntimeError):
@@ -75,6 +75,7 @@ _lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P,
 _lib.veda_estimator_grad.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _I, _P] + [_P] * 8 + [_P, _P, _P]
 _lib.veda_estimator_grad_ws_bytes.argtypes = [_LP, _I, _I, _I, _I]
 _lib.veda_estimator_grad_ws_bytes.restype = ctypes.c_size_t
+_lib.veda_output_sq_error.argtypes = [_LP, _P, _P, _P, _P]
 _lib.veda_check_status.argtypes = [_LP, _P]
 _lib.veda_selftest_wait_timeout.argtypes = [_LP, ctypes.c_uint32, _P]
 _lib.veda_last_error.restype = ctypes.c_char_p
@@ -226,6 +227,10 @@ def veda_estimator_grad(layer: Layer, dq, dk, weights: Sequence[torch.Tensor], h
                                     float(scale), _host_i32(heads_sel), len(heads_sel), _ptr(qtile_rows),
                                     int(n_rows), _ptr(tilemap), *[_ptr(t) for t in grads], _ptr(loss), _ptr(ws),
                                     _stream(stream)))
+
+
+def veda_output_sq_error(layer: Layer, a: torch.Tensor, b: torch.Tensor, err: torch.Tensor, stream=None):
+    _check(_lib.veda_output_sq_error(layer.ref, _ptr(a), _ptr(b), _ptr(err), _stream(stream)))
 
 
 def veda_check_status(layer: Layer, stream=None):

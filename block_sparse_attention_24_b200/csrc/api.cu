@@ -362,6 +362,15 @@ int veda_estimator_grad(const veda_layer* L, const float* dq, const float* dk, c
                       "veda_estimator_grad");
 }
 
+int veda_output_sq_error(const veda_layer* L, const void* a, const void* b, float* err, cudaStream_t stream) {
+  veda::LayerGeom g;
+  VEDA_TRY(build_geom(L, &g));
+  VEDA_TRY(check_ptr(a, "a"));
+  VEDA_TRY(check_ptr(b, "b"));
+  VEDA_TRY(check_ptr(err, "err"));
+  return after_launch(veda::launch_output_sq_error(g, a, b, err, stream), "veda_output_sq_error");
+}
+
 int veda_check_status(const veda_layer* L, cudaStream_t stream) {
   if (!L || !L->dev_status) return fail(VEDA_ERR_INVALID_ARG, "layer or dev_status is NULL");
   cudaError_t e = cudaStreamSynchronize(stream);

@@ -389,6 +389,7 @@ cudaError_t launch_estimator_grad(const LayerGeom& g, const float* dq, const flo
                                   float* const gw[8], int hidden, int out_dim, float scale, const int32_t* heads_sel,
                                   int n_heads_sel, const int32_t* rows, int n_rows, const float* tilemap,
                                   float* loss, float* ws, cudaStream_t s);
+cudaError_t launch_output_sq_error(const LayerGeom& g, const void* a, const void* b, float* err, cudaStream_t s);
 cudaError_t launch_tile_scores(const LayerGeom& g, const float* dq, const float* dk, const float* w1q,
                                const float* b1q, const float* w2q, const float* b2q, const float* w1k,
                                const float* b1k, const float* w2k, const float* b2k, int hidden, int out_dim,

@@ -226,6 +226,14 @@ int veda_estimator_grad(const veda_layer* L, const float* dq, const float* dk,
                         float* g_w1k, float* g_b1k, float* g_w2k, float* g_b2k,
                         float* loss, float* ws, cudaStream_t stream);
 
+/* Calibration metric of the head-aware tiling search (Veda summary 2.2:
+ * tilings are chosen per head, offline, to fit each head's locality):
+ * err[h] (device fp32 [heads]) = sum over batch, tokens and channels of
+ * (a - b)^2 for head h, with a and b [B,N,heads,d] bf16 attention outputs in
+ * the original token order (e.g. full attention and the tile-skipping
+ * output under one candidate tiling). Fixed-order reduction. */
+int veda_output_sq_error(const veda_layer* L, const void* a, const void* b, float* err, cudaStream_t stream);
+
 /* Diagnostic (no counterpart on the pages): launches one thread that waits,
  * through the bounded wait every pipeline kernel uses, on a barrier nothing
  * arrives on. After limit_ms (1..10000) the wait gives up and records
