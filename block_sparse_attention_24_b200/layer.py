@@ -104,10 +104,12 @@ class VedaLayer:
                          stream=stream)
         veda_topk_mask(L, self.scores, self.k, self.k_cap, self.idx, self.mask, stream=stream)
 
-    def attend(self, stream=None):
+    def attend(self, stream=None, out: Optional[torch.Tensor] = None):
+        """Sparse attention and the inverse permutation into `out` (default:
+        the layer's own output buffer)."""
         veda_sparse_attn(self.L, self.qp, self.kp, self.vp, self.idx, self.k, self.k_cap, self.attn_scale, self.op,
                          stream=stream)
-        veda_permute(self.L, self.o, self.op, inverse=True, stream=stream)
+        veda_permute(self.L, self.o if out is None else out, self.op, inverse=True, stream=stream)
 
     def distill(self, stream=None):
         if self.maps is None:
@@ -151,3 +153,63 @@ def device_weights(np_weights, device) -> Dict[str, torch.Tensor]:
     """The same per-head MLP for query and key descriptors (w1, b1, w2, b2)."""
     w1, b1, w2, b2 = (torch.from_numpy(a).to(device) for a in np_weights)
     return {"w1q": w1, "b1q": b1, "w2q": w2, "b2q": b2, "w1k": w1, "b1k": b1, "w2k": w2, "b2k": b2}
+
+
+class HostPipeline:
+    """Runs a layer over host-resident inputs with the copies hidden behind
+    the kernels: while step i computes, the host->device copy of step i+1's
+    Q, K, V and the device->host copy of step i-1's output run on two copy
+    streams (PCIe moves both directions at once). Two device input sets and
+    two device output buffers alternate; events order every reuse. Each step
+    still copies its own inputs in and its own output (and KL) out."""
+
+    def __init__(self, layer: VedaLayer, q_like: torch.Tensor):
+        dev = layer.device
+        self.layer = layer
+        self.inputs = [[torch.empty_like(q_like, device=dev) for _ in range(3)] for _ in range(2)]
+        self.outputs = [torch.empty_like(layer.o) for _ in range(2)]
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.compute_done = [None, None]   # compute of the step that last used slot s
+        self.d2h_done = [None, None]       # output copy of the step that last used slot s
+
+    def run(self, host_qkv, host_out, host_kl=None, steps: int = 1):
+        """host_qkv: pinned (q, k, v) host tensors; host_out: pinned host
+        tensor of the output's shape (and host_kl of kl_out's, optional),
+        rewritten every step. Returns when every copy has been enqueued."""
+        comp = torch.cuda.current_stream(self.layer.device)
+        for i in range(steps):
+            s = i % 2
+            dq, dk, dv = self.inputs[s]
+            if self.compute_done[s] is not None:
+                self.h2d.wait_event(self.compute_done[s])     # slot s's inputs are free again
+            with torch.cuda.stream(self.h2d):
+                for dst, src in zip((dq, dk, dv), host_qkv):
+                    dst.copy_(src, non_blocking=True)
+                loaded = torch.cuda.Event()
+                loaded.record(self.h2d)
+            comp.wait_event(loaded)
+            if self.d2h_done[s] is not None:
+                comp.wait_event(self.d2h_done[s])             # slot s's output was copied out
+            layer = self.layer
+            layer.front(dq, dk, dv)
+            layer.attend(out=self.outputs[s])
+            layer.distill()
+            if host_kl is not None and layer.maps is not None:
+                host_kl.copy_(layer.kl_out, non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(comp)
+            self.compute_done[s] = done
+            self.d2h.wait_event(done)
+            with torch.cuda.stream(self.d2h):
+                host_out.copy_(self.outputs[s], non_blocking=True)
+                copied = torch.cuda.Event()
+                copied.record(self.d2h)
+            self.d2h_done[s] = copied
+
+    def wait(self):
+        """Make the current stream wait for every copy issued so far."""
+        comp = torch.cuda.current_stream(self.layer.device)
+        for e in self.d2h_done:
+            if e is not None:
+                comp.wait_event(e)
