@@ -264,12 +264,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "model": "none (one attention layer, synthetic activations)",
-                   "global_batch": w.B * world, "seq_len": w.N, "heads": w.heads, "head_dim": w.d,
-                   "tile": w.tile, "keep": w.keep, "sparsity": round(1 - kept / allp, 4),
-                   "tilemap": {"heads": list(w.tilemap_heads), "query_tiles_per_head": int(layer.maps.n_rows)},
-                   "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
-                   "l2": l2_note(q)},
+        "config": bench_config(w, world, round(1 - kept / allp, 4), int(layer.maps.n_rows)),
         "attn_ms": round(attn_ms, 3), "attn_tflops": round(attn_tflops, 1),
         "attn_frac_of_burst_peak": round(attn_tflops / burst, 4),
         "dense_ms": round(dense_ms, 3), "speedup_vs_dense": round(dense_ms / attn_ms, 2),
@@ -360,14 +355,31 @@ def run_e2e(V, L, layer, q, k, v, device, eff_flops, args):
             "copies": "overlapped with the kernels of the neighbouring steps (two copy streams)"}
 
 
-def l2_note(q) -> str:
-    """How the timed region avoids L2 reuse between steps: the inputs are
-    larger than the 126 MB L2, or (small layers) they are not and the note
-    says so."""
-    mb = q.numel() * q.element_size() / 1e6
-    if mb > 126:
-        return f"inputs larger than L2 (each of Q/K/V is {mb:.0f} MB)"
-    return f"inputs fit in L2 (each of Q/K/V is {mb:.0f} MB); parity-size layer, not the benchmark layer"
+def bench_config(w, world, sparsity, map_rows) -> dict:
+    """The workload description both arms print."""
+    qkv_mb = w.B * w.N * w.heads * w.d * 2 / 1e6
+    return {"workload": w.name, "model": "none (one attention layer, synthetic activations)",
+            "global_batch": w.B * world, "seq_len": w.N, "heads": w.heads, "head_dim": w.d,
+            "tile": w.tile, "keep": w.keep, "sparsity": sparsity,
+            "tilemap": {"heads": list(w.tilemap_heads), "query_tiles_per_head": int(map_rows)},
+            "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
+            "l2": (f"inputs larger than L2 (each of Q/K/V is {qkv_mb:.0f} MB)" if qkv_mb > 126 else
+                   f"inputs fit in L2 (each of Q/K/V is {qkv_mb:.0f} MB); parity-size layer, not the benchmark layer")}
+
+
+def layout_sparsity(w) -> float:
+    """Sparsity from the layout alone: exact when no head's T is padded (every
+    tile full, so kept pairs = nt * k * tile^2 per head), else the nominal
+    1 - keep."""
+    kept = allp = 0
+    for pt, ph, pw in w.tilings:
+        if w.T % pt:
+            return round(1 - w.keep, 4)
+        nt = (w.T // pt) * (w.H // ph) * (w.W // pw)
+        kk = max(1, int(math.floor(w.keep * nt + 0.5)))
+        kept += nt * kk
+        allp += nt * nt
+    return round(1 - kept / allp, 4)
 
 
 def kernel_source_hash() -> str:
@@ -502,7 +514,7 @@ def run_reference(args, world, rank, local):
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": w.name, "keep": w.keep, "tile": w.tile},
+        "config": bench_config(w, world, layout_sparsity(w), MAP_ROWS),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                          "sample": f"per step: oracle front end for head {h} + sparse attention on "
                                    f"~{tiles / max(1, args.steps):.0f} seeded query tiles"},
