@@ -38,7 +38,7 @@ import synth  # noqa: E402
 METRIC = "block-sparse attn ms/layer & effective TFLOP/s at 90% sparsity vs dense path"
 UNIT = "TFLOP/s"
 MAP_ROWS = 120          # query tiles per tile-map head (10% of 1200: sparse supervision)
-KERNELS_PER_STEP = 11   # 2 permute+TripPool, permute V, MLP + score GEMM, top-k, attention, unpermute, map, KL rows, KL mean
+KERNELS_PER_STEP = 12   # 2 permute+TripPool, permute V, MLP + score GEMM, top-k, attention, unpermute, map (2 passes), KL rows, KL mean
 
 
 # ------------------------------------------------------------------ ranks

@@ -27,7 +27,8 @@ VEDA_ERR_BAD_INDEX = -5
 
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
-            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_check_status",
+            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes",
+            "veda_check_status",
             "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_output_sq_error", "veda_selftest_wait_timeout", "veda_last_error")
 
 
@@ -71,7 +72,9 @@ _lib.veda_tile_scores_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_topk_mask.argtypes = [_LP, _P, _P, _I, _P, _P, _P]
 _lib.veda_tile_scores_topk.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _P, _P, _P, _P]
 _lib.veda_sparse_attn.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
-_lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P, _P, _P, _P, _P]
+_lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P, _P, _P, _P, _P, _P]
+_lib.veda_full_attn_tilemax_ws_bytes.argtypes = [_LP, _I, _I]
+_lib.veda_full_attn_tilemax_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_estimator_grad.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _I, _P] + [_P] * 8 + [_P, _P, _P]
 _lib.veda_estimator_grad_ws_bytes.argtypes = [_LP, _I, _I, _I, _I]
 _lib.veda_estimator_grad_ws_bytes.restype = ctypes.c_size_t
@@ -81,7 +84,8 @@ _lib.veda_selftest_wait_timeout.argtypes = [_LP, ctypes.c_uint32, _P]
 _lib.veda_last_error.restype = ctypes.c_char_p
 for _name in EXPORTED:
     getattr(_lib, _name)
-    if _name not in ("veda_last_error", "veda_tile_scores_ws_bytes", "veda_estimator_grad_ws_bytes"):
+    if _name not in ("veda_last_error", "veda_tile_scores_ws_bytes", "veda_estimator_grad_ws_bytes",
+                     "veda_full_attn_tilemax_ws_bytes"):
         getattr(_lib, _name).restype = ctypes.c_int
 
 
@@ -208,10 +212,14 @@ def veda_sparse_attn(layer: Layer, qp, kp, vp, idx: Optional[torch.Tensor], k: O
 def veda_full_attn_tilemax(layer: Layer, qp, kp, heads_sel: Sequence[int], qtile_rows: Optional[torch.Tensor],
                            n_rows: int, scale: float, tilemap: torch.Tensor, lse: Optional[torch.Tensor] = None,
                            scores: Optional[torch.Tensor] = None, kl_rows: Optional[torch.Tensor] = None,
-                           kl_out: Optional[torch.Tensor] = None, stream=None):
+                           kl_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
     _check(_lib.veda_full_attn_tilemax(layer.ref, _ptr(qp), _ptr(kp), _host_i32(heads_sel), len(heads_sel),
                                        _ptr(qtile_rows), int(n_rows), float(scale), _ptr(tilemap), _ptr(lse),
-                                       _ptr(scores), _ptr(kl_rows), _ptr(kl_out), _stream(stream)))
+                                       _ptr(scores), _ptr(kl_rows), _ptr(kl_out), _ptr(ws), _stream(stream)))
+
+
+def veda_full_attn_tilemax_ws_bytes(layer: Layer, n_heads_sel: int, n_rows: int) -> int:
+    return int(_lib.veda_full_attn_tilemax_ws_bytes(layer.ref, n_heads_sel, n_rows))
 
 
 def veda_estimator_grad_ws_bytes(layer: Layer, n_heads_sel: int, n_rows: int, hidden: int, out_dim: int) -> int:

@@ -275,10 +275,16 @@ int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const 
                       "veda_sparse_attn");
 }
 
+size_t veda_full_attn_tilemax_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows) {
+  veda::LayerGeom g;
+  if (build_geom(L, &g) != VEDA_OK || n_heads_sel < 1 || n_rows < 1) return 0;
+  return veda::tilemax_ws_bytes(n_heads_sel, n_rows, g.tile);
+}
+
 int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp, const int32_t* heads_sel,
                            int32_t n_heads_sel, const int32_t* qtile_rows, int32_t n_rows, float scale,
                            float* tilemap, float* lse, const float* scores, float* kl_rows, float* kl_out,
-                           cudaStream_t stream) {
+                           float* ws, cudaStream_t stream) {
   veda::LayerGeom g;
   VEDA_TRY(build_geom(L, &g));
   if (g.B != 1) return fail(VEDA_ERR_UNSUPPORTED, "tile map: only B == 1 layers are accepted");
@@ -286,6 +292,7 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp, 
   VEDA_TRY(check_ptr(kp, "kp"));
   VEDA_TRY(check_ptr(tilemap, "tilemap"));
   if (lse) VEDA_TRY(check_ptr(lse, "lse"));
+  if (ws) VEDA_TRY(check_ptr(ws, "ws"));
   if (qtile_rows) VEDA_TRY(check_ptr(qtile_rows, "qtile_rows"));
   if (!heads_sel || n_heads_sel < 1 || n_heads_sel > VEDA_MAX_HEADS)
     return fail(VEDA_ERR_INVALID_ARG, "heads_sel must list 1..%d heads", VEDA_MAX_HEADS);
@@ -304,7 +311,7 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp, 
     VEDA_TRY(check_ptr(kl_out, "kl_out"));
   }
   return after_launch(veda::launch_tilemax(g, qp, kp, heads_sel, n_heads_sel, qtile_rows, n_rows, scale, tilemap,
-                                           lse, scores, scores ? kl_rows : nullptr, scores ? kl_out : nullptr,
+                                           lse, scores, scores ? kl_rows : nullptr, scores ? kl_out : nullptr, ws,
                                            stream),
                       "veda_full_attn_tilemax");
 }

@@ -11,6 +11,8 @@
 //           softmax probability over the tile region.
 // A second kernel turns map rows and score rows into KL values, a third
 // averages them in a fixed order.
+#include <climits>
+
 #include "veda_internal.cuh"
 
 namespace veda {
@@ -20,6 +22,7 @@ constexpr int BM = 128, BN = 128;
 constexpr int KST = 3;                 // K ring stages
 constexpr uint32_t TMEM_COLS = 512;    // S buffers: row-block r, buffer b at (2r + b) * 128
 constexpr int NUM_THREADS = 384;
+constexpr int MAP_MAX_SPLIT = 8;       // most CTAs one row pair's key range is split over
 // softmax warpgroups 216 registers, producer/MMA warpgroup 72:
 // 2*128*216 + 128*72 = 64,512 = the 384*168 the launch reserves (208/88
 // removes the producer warps' few spills but measured 10% slower)
@@ -42,6 +45,9 @@ struct MapLayout {
 
 struct MapParams {
   float scale_log2;
+  int mode;             // 0: both passes; 1: pass 1 only, partial sums to ws; 2: pass 2 only, from ws
+  int n_split;          // CTAs sharing one row pair's key range (blockIdx.z); 1 for mode 0
+  float2* ws;           // [n_heads_sel][n_rows][tile][n_split] (reference m, sum l) in log2 units
   int n_rows;
   const int32_t* rows;  // [n_heads_sel, n_rows] or NULL
   float* tilemap;       // [n_heads_sel, n_rows, nt_cap]
@@ -129,7 +135,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int nt = hg.nt;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_kb = (nt * TILE + BN - 1) / BN;
-  const int iters = 2 * n_kb;
+  // this CTA's share of the key blocks (all of them unless the key range is
+  // split over blockIdx.z)
+  const int split = blockIdx.z;
+  const int kb_begin = (int)((long long)n_kb * split / prm.n_split);
+  const int kb_end = (int)((long long)n_kb * (split + 1) / prm.n_split);
+  const int nkb = kb_end - kb_begin;
+  const int iters = (prm.mode == 0 ? 2 : 1) * nkb;
 
   // selected query tiles: entry (2*blockIdx.x + r)*NSUB + s of the row list
   int qt[2][NSUB];
@@ -201,7 +213,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int st = it % KST;
         if (it >= KST && !mbar_wait(k_empty + st, ((it - KST) / KST) & 1, abort_flag, g.dev_status)) break;
         mbar_expect_tx(k_full + st, Lay::KB);
-        const int kb = it % n_kb;
+        const int kb = kb_begin + it % nkb;
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
           tma_load_3d(smem + Lay::OFF_K + st * Lay::KB + bx * BN * 128, &tmK, k_full + st, bx * 64, kb * BN, bh);
@@ -255,6 +267,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float C = prm.scale_log2;
     const uint64_t C2 = f2(C, C);
     float m = -INFINITY, l = 0.f, lse2 = 0.f;
+    const int e_row = (2 * blockIdx.x + r) * NSUB + qs;  // this row's entry in the row list
+    // partial (reference, sum) of row `row` of entry e_row from split sp
+    auto part_ws = [&](int sp) -> float2* {
+      return prm.ws + (((long long)hs * prm.n_rows + e_row) * TILE + (row % TILE)) * prm.n_split + sp;
+    };
+    if (prm.mode == 2 && rb_valid[r] && e_row < prm.n_rows) {
+      // combine the splits' partial sums in a fixed order: every split's CTA
+      // gets the same log-sum-exp
+      float M = -INFINITY;
+      for (int sp = 0; sp < prm.n_split; ++sp) M = fmaxf(M, part_ws(sp)->x);
+      float L = 0.f;
+      for (int sp = 0; sp < prm.n_split; ++sp) {
+        const float2 pr = *part_ws(sp);
+        if (pr.y > 0.f) L += pr.y * fast_exp2(pr.x - M);
+      }
+      lse2 = M + __log2f(L);
+      if (prm.lse && split == 0)
+        prm.lse[((long long)hs * prm.n_rows + e_row) * TILE + (row % TILE)] = row_valid ? lse2 * 0.69314718055994531f : 0.f;
+    }
     for (int it = 0; it < (rb_valid[r] ? iters : 0); ++it) {
       const int sb = 2 * r + (it & 1);
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, (it >> 1) & 1, abort_flag, g.dev_status))) break;
@@ -263,8 +294,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld128(lane_addr + sb * BN, u);
       tc_fence_before();
       mbar_arrive(s_free + sb);  // S buffer may be overwritten now
-      const int kb = it % n_kb;
-      const bool pass2 = it >= n_kb;
+      const int kb = kb_begin + it % nkb;
+      const bool pass2 = prm.mode == 2 || (prm.mode == 0 && it >= nkb);
 #pragma unroll
       for (int uu = 0; uu < NSUB; ++uu) {
         const int kt = kb * NSUB + uu;
@@ -302,13 +333,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0 && kt < nt && v > -INFINITY) atomicMax(part + (r * NSUB + qs) * g.nt_cap + kt, ord_f32(v));
         }
       }
-      if (it == n_kb - 1) {
+      if (prm.mode == 0 && it == nkb - 1) {
         lse2 = m + __log2f(l);
-        const int e = (2 * blockIdx.x + r) * NSUB + qs;
-        if (prm.lse && e < prm.n_rows)
-          prm.lse[((long long)hs * prm.n_rows + e) * TILE + (row % TILE)] = row_valid ? lse2 * 0.69314718055994531f : 0.f;
+        if (prm.lse && e_row < prm.n_rows)
+          prm.lse[((long long)hs * prm.n_rows + e_row) * TILE + (row % TILE)] = row_valid ? lse2 * 0.69314718055994531f : 0.f;
       }
     }
+    if (prm.mode == 1 && e_row < prm.n_rows) *part_ws(split) = make_float2(m, l);
     tc_fence_before();
   }
   __syncthreads();
@@ -316,8 +347,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
-  // write the map rows
-  if (!*abort_flag) {
+  // write the map rows: this CTA's key tiles (the last split also writes
+  // the zero columns past nt)
+  const int kt_begin = kb_begin * NSUB;
+  const int kt_end = split == prm.n_split - 1 ? g.nt_cap : kb_end * NSUB;
+  if (!*abort_flag && prm.mode != 1) {
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -325,7 +359,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int e = (2 * blockIdx.x + r) * NSUB + s;
         if (e >= prm.n_rows) continue;
         float* out = prm.tilemap + ((long long)hs * prm.n_rows + e) * g.nt_cap;
-        for (int b = threadIdx.x; b < g.nt_cap; b += NUM_THREADS) {
+        for (int b = kt_begin + threadIdx.x; b < kt_end; b += NUM_THREADS) {
           const uint32_t k = part[(r * NSUB + s) * g.nt_cap + b];
           out[b] = (b < nt && k != 0u && qv[r][s]) ? fast_exp2(unord_f32(k)) : 0.f;
         }
@@ -396,7 +430,7 @@ __global__ void kl_mean_kernel(const float* __restrict__ kl_rows, int n_heads_se
 }
 
 template <int D, int TILE>
-cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, const MapParams& prm, int n_heads_sel,
+cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, MapParams prm, int n_heads_sel,
                          cudaStream_t s) {
   CUtensorMap tq, tk;
   const uint64_t rows = (uint64_t)g.n_cap, planes = (uint64_t)g.B * g.heads;
@@ -408,17 +442,61 @@ cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, con
   if (smem > 232448) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((prm.n_rows + 2 * NSUB - 1) / (2 * NSUB), n_heads_sel, 1);
-  kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, prm);
+  const int pairs = (prm.n_rows + 2 * NSUB - 1) / (2 * NSUB);
+  // With a workspace, split each row pair's key range over n_split CTAs when
+  // that fills the SMs' waves noticeably better (one CTA per SM): pass 1
+  // writes partial sums, pass 2 combines them and builds its own key tiles.
+  int n_split = 1;
+  if (prm.ws) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int n_kb_min = INT_MAX;
+    for (int i = 0; i < n_heads_sel; ++i) {
+      const int nt = g.h[prm.heads_sel[i]].nt;
+      const int nkb = (nt * TILE + BN - 1) / BN;
+      n_kb_min = nkb < n_kb_min ? nkb : n_kb_min;
+    }
+    const long long base = (long long)pairs * n_heads_sel;
+    auto fill = [&](int sp) {
+      const long long ctas = base * sp, waves = (ctas + sms - 1) / sms;
+      return (double)ctas / (double)(waves * sms);
+    };
+    double best = fill(1);
+    for (int sp = 2; sp <= MAP_MAX_SPLIT && n_kb_min / sp >= 4; ++sp)
+      if (fill(sp) > best + 0.05) {
+        best = fill(sp);
+        n_split = sp;
+      }
+  }
+  if (n_split == 1) {
+    prm.mode = 0;
+    prm.n_split = 1;
+    kern<<<dim3(pairs, n_heads_sel, 1), NUM_THREADS, smem, s>>>(g, tq, tk, prm);
+    return cudaGetLastError();
+  }
+  prm.n_split = n_split;
+  prm.mode = 1;
+  kern<<<dim3(pairs, n_heads_sel, n_split), NUM_THREADS, smem, s>>>(g, tq, tk, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  prm.mode = 2;
+  kern<<<dim3(pairs, n_heads_sel, n_split), NUM_THREADS, smem, s>>>(g, tq, tk, prm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile) {
+  return (size_t)n_heads_sel * n_rows * tile * MAP_MAX_SPLIT * sizeof(float2);
+}
+
 cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, const int32_t* heads_sel,
                            int n_heads_sel, const int32_t* rows, int n_rows, float scale, float* tilemap, float* lse,
-                           const float* scores, float* kl_rows, float* kl_out, cudaStream_t s) {
+                           const float* scores, float* kl_rows, float* kl_out, float* ws, cudaStream_t s) {
   MapParams prm;
+  prm.mode = 0;
+  prm.n_split = 1;
+  prm.ws = reinterpret_cast<float2*>(ws);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.n_rows = n_rows;
   prm.rows = rows;

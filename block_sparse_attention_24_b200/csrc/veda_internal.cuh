@@ -399,9 +399,10 @@ cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int3
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, int k_cap, float scale, void* op, float* lse,
                                cudaStream_t s);
+size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile);
 cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, const int32_t* heads_sel,
-                           int n_heads_sel, const int32_t* rows, int n_rows, float scale, float* tilemap,
-                           float* lse, const float* scores, float* kl_rows, float* kl_out, cudaStream_t s);
+                           int n_heads_sel, const int32_t* rows, int n_rows, float scale, float* tilemap, float* lse,
+                           const float* scores, float* kl_rows, float* kl_out, float* ws, cudaStream_t s);
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                                    uint32_t box0, uint32_t box1);

@@ -17,8 +17,9 @@ from typing import Dict, List, Optional, Sequence
 
 import torch
 
-from . import (Layer, veda_estimator_grad, veda_estimator_grad_ws_bytes, veda_full_attn_tilemax, veda_permute,
-               veda_permute_trippool, veda_sparse_attn, veda_tile_scores, veda_tile_scores_ws_bytes, veda_topk_mask)
+from . import (Layer, veda_estimator_grad, veda_estimator_grad_ws_bytes, veda_full_attn_tilemax,
+               veda_full_attn_tilemax_ws_bytes, veda_permute, veda_permute_trippool, veda_sparse_attn, veda_tile_scores,
+               veda_tile_scores_ws_bytes, veda_topk_mask)
 
 
 def k_from_keep(keep: float, nt: int) -> int:
@@ -71,6 +72,7 @@ class VedaLayer:
             self.map_lse = torch.empty((nh, maps.n_rows, layer.tile), **f32)
             self.kl_rows = torch.empty((nh, maps.n_rows), **f32)
             self.kl_out = torch.zeros(4, **f32)
+            self.map_ws = torch.empty(veda_full_attn_tilemax_ws_bytes(layer, nh, maps.n_rows) // 4, **f32)
 
     def effective_flops(self, idx_host=None) -> float:
         """4*d*sum of kept valid (query, key) token pairs over all heads, from
@@ -116,7 +118,7 @@ class VedaLayer:
             return
         m = self.maps
         veda_full_attn_tilemax(self.L, self.qp, self.kp, m.heads, m.rows, m.n_rows, self.attn_scale, self.tilemap,
-                               self.map_lse, self.scores, self.kl_rows, self.kl_out, stream=stream)
+                               self.map_lse, self.scores, self.kl_rows, self.kl_out, ws=self.map_ws, stream=stream)
 
     def estimator_grad(self, stream=None):
         """Weight gradient of the distillation loss on this step's tile-map

@@ -189,12 +189,17 @@ int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const 
  * of] veda_tile_scores output) is not NULL, kl_rows [n_heads_sel, n_rows]
  * receives KL(t || softmax(scores row)) with t the tile-map row normalised to
  * sum 1, and *kl_out (device fp32) their mean over rows, then heads.
- * Only B == 1 layers are accepted. */
+ * ws (may be NULL): veda_full_attn_tilemax_ws_bytes(...) bytes of device
+ * scratch; with it the call may split each pair of query tiles' key range
+ * over several CTAs (two launches: partial sums, then their fixed-order
+ * combination) so that small maps fill every SM; results are the same up to
+ * fp32 rounding of the log-sum-exp. Only B == 1 layers are accepted. */
+size_t veda_full_attn_tilemax_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows);
 int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp,
                            const int32_t* heads_sel, int32_t n_heads_sel,
                            const int32_t* qtile_rows, int32_t n_rows, float scale,
                            float* tilemap, float* lse, const float* scores,
-                           float* kl_rows, float* kl_out, cudaStream_t stream);
+                           float* kl_rows, float* kl_out, float* ws, cudaStream_t stream);
 
 /* Estimator training (Veda summary 2.1, Optimization: the head-specific
  * projections are trained with the row-wise KL against the tile map, with

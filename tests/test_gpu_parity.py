@@ -456,3 +456,45 @@ def test_tilemap_all_rows_default_list():
     for s, h in enumerate([1, 0]):
         M, _ = O.full_tilemap(f64(qp)[0, h], f64(kp)[0, h], lays[h]["lens"], w.tile, 0.125)
         _row_rel(gm[s], M)
+
+
+@pytest.mark.parametrize("idx,heads,n_rows", [(1, [3, 7], 6), (2, [0], 5), (4, [1, 5], 9)])
+def test_tilemap_split_key_range(idx, heads, n_rows):
+    """With a workspace the map may split each row pair's key range over
+    several CTAs (partial sums, then a fixed-order combination): same map,
+    log-sum-exp and KL as the single-CTA path, and the oracle's values on the
+    rows checked. Layers: 24,576 tokens with 64-token tiles, 80,640 tokens
+    with padded T, 65,280 tokens."""
+    w = synth.config(idx)
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, k, _ = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    kp, _ = _permuted(L, w, k)
+    rng = np.random.default_rng(11)
+    rows = np.stack([np.sort(rng.choice(lays[h]["nt"], n_rows, replace=False)) for h in heads]).astype(np.int32)
+    rows_d = torch.from_numpy(rows).to(DEV)
+    scores = torch.from_numpy(rng.standard_normal((1, w.heads, nt_cap, nt_cap)).astype(np.float32)).to(DEV)
+    scale = 1 / math.sqrt(w.d)
+    out = {}
+    for use_ws in (False, True):
+        tm = torch.full((len(heads), n_rows, nt_cap), 7.0, dtype=torch.float32, device=DEV)
+        lse = torch.full((len(heads), n_rows, w.tile), 7.0, dtype=torch.float32, device=DEV)
+        klr = torch.empty((len(heads), n_rows), dtype=torch.float32, device=DEV)
+        klo = torch.empty(4, dtype=torch.float32, device=DEV)
+        ws = None
+        if use_ws:
+            ws = torch.empty(V.veda_full_attn_tilemax_ws_bytes(L, len(heads), n_rows) // 4, dtype=torch.float32,
+                             device=DEV)
+        V.veda_full_attn_tilemax(L, qp, kp, heads, rows_d, n_rows, scale, tm, lse, scores, klr, klo, ws=ws)
+        V.veda_check_status(L)
+        out[use_ws] = [t.cpu().double().numpy() for t in (tm, lse, klr, klo[:1])]
+    for a, b in zip(out[False], out[True]):
+        np.testing.assert_allclose(b, a, rtol=1e-5, atol=1e-30)
+    gm = out[True][0]
+    for s, h in enumerate(heads):
+        nt = lays[h]["nt"]
+        pick = [0, n_rows - 1]
+        M, _ = O.full_tilemap(f64(qp)[0, h], f64(kp)[0, h], lays[h]["lens"], w.tile, scale, rows[s, pick])
+        _row_rel(gm[s, pick, :nt], M)
+        assert not gm[s, :, nt:].any()
