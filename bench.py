@@ -196,8 +196,10 @@ def run_ours(args, world, rank, local):
     eff_flops = 4.0 * L.d * kept
     n_stage = len(layer.STAGES)
 
-    # timed region: whole steps, with events around each stage on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    # timed region: whole steps (layer.forward), with events at the stage
+    # boundaries on the launching stream
+    names = ("start", "front", "attn0", "attn1", "unpermute", "end")
+    ev = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize(device)
     if True:  # the timed region
@@ -206,17 +208,7 @@ def run_ours(args, world, rank, local):
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for s in range(args.steps):
-            e = ev[s]
-            e[0].record(stream)
-            layer.front(q, k, v)
-            e[1].record(stream)
-            V.veda_sparse_attn(L, layer.qp, layer.kp, layer.vp, layer.idx, layer.k, layer.k_cap, layer.attn_scale,
-                               layer.op)
-            e[2].record(stream)
-            V.veda_permute(L, layer.o, layer.op, inverse=True)
-            e[3].record(stream)
-            layer.distill()
-            e[4].record(stream)
+            layer.forward(q, k, v, marks=ev[s])
         t1.record(stream)
         torch.cuda.synchronize(device)
         host_t1 = datetime.datetime.now()
@@ -224,10 +216,10 @@ def run_ours(args, world, rank, local):
     elapsed = t0.elapsed_time(t1) / 1e3
     elapsed = max_over_ranks(elapsed, device)
     V.veda_check_status(L)
-    front_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    unperm_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
-    map_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in ev)
+    front_ms = statistics.mean(e["start"].elapsed_time(e["front"]) for e in ev)
+    attn_ms = statistics.mean(e["attn0"].elapsed_time(e["attn1"]) for e in ev)
+    unperm_ms = statistics.mean(e["attn1"].elapsed_time(e["unpermute"]) for e in ev)
+    tail_ms = statistics.mean(e["unpermute"].elapsed_time(e["end"]) for e in ev)
     clk.__exit__(None, None, None)
     clocks = clk.summary(host_t0, host_t1)
 
@@ -270,7 +262,7 @@ def run_ours(args, world, rank, local):
         "dense_ms": round(dense_ms, 3), "speedup_vs_dense": round(dense_ms / attn_ms, 2),
         "layer_ms": round(front_ms + attn_ms + unperm_ms, 3),
         "stage_ms": {**stage_ms, "front_end": round(front_ms, 3), "sparse_attn": round(attn_ms, 3),
-                     "unpermute": round(unperm_ms, 3), "tilemap_kl": round(map_ms, 3)},
+                     "unpermute": round(unperm_ms, 3), "tilemap_kl": round(tail_ms, 3)},
         "estimator_grad_ms": grad_ms,
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": sustained, "unit": UNIT,
                      "frac": round(attn_tflops / sustained, 4), "traffic": traffic,

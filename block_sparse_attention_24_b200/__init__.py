@@ -27,7 +27,7 @@ VEDA_ERR_BAD_INDEX = -5
 
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
-            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes",
+            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes", "veda_tilemap_kl",
             "veda_check_status",
             "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_output_sq_error", "veda_selftest_wait_timeout", "veda_last_error")
 
@@ -74,6 +74,7 @@ _lib.veda_tile_scores_topk.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _
 _lib.veda_sparse_attn.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
 _lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P, _P, _P, _P, _P, _P]
 _lib.veda_full_attn_tilemax_ws_bytes.argtypes = [_LP, _I, _I]
+_lib.veda_tilemap_kl.argtypes = [_LP, _P, _I, _P, _I, _P, _P, _P, _P, _P]
 _lib.veda_full_attn_tilemax_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_estimator_grad.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _I, _P] + [_P] * 8 + [_P, _P, _P]
 _lib.veda_estimator_grad_ws_bytes.argtypes = [_LP, _I, _I, _I, _I]
@@ -216,6 +217,13 @@ def veda_full_attn_tilemax(layer: Layer, qp, kp, heads_sel: Sequence[int], qtile
     _check(_lib.veda_full_attn_tilemax(layer.ref, _ptr(qp), _ptr(kp), _host_i32(heads_sel), len(heads_sel),
                                        _ptr(qtile_rows), int(n_rows), float(scale), _ptr(tilemap), _ptr(lse),
                                        _ptr(scores), _ptr(kl_rows), _ptr(kl_out), _ptr(ws), _stream(stream)))
+
+
+def veda_tilemap_kl(layer: Layer, heads_sel: Sequence[int], qtile_rows: Optional[torch.Tensor], n_rows: int,
+                    tilemap: torch.Tensor, scores: torch.Tensor, kl_rows: torch.Tensor, kl_out: torch.Tensor,
+                    stream=None):
+    _check(_lib.veda_tilemap_kl(layer.ref, _host_i32(heads_sel), len(heads_sel), _ptr(qtile_rows), int(n_rows),
+                                _ptr(tilemap), _ptr(scores), _ptr(kl_rows), _ptr(kl_out), _stream(stream)))
 
 
 def veda_full_attn_tilemax_ws_bytes(layer: Layer, n_heads_sel: int, n_rows: int) -> int:

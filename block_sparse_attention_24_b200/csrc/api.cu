@@ -316,6 +316,32 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp, 
                       "veda_full_attn_tilemax");
 }
 
+int veda_tilemap_kl(const veda_layer* L, const int32_t* heads_sel, int32_t n_heads_sel, const int32_t* qtile_rows,
+                    int32_t n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,
+                    cudaStream_t stream) {
+  veda::LayerGeom g;
+  VEDA_TRY(build_geom(L, &g));
+  if (g.B != 1) return fail(VEDA_ERR_UNSUPPORTED, "tile map KL: only B == 1 layers are accepted");
+  VEDA_TRY(check_ptr(tilemap, "tilemap"));
+  VEDA_TRY(check_ptr(scores, "scores"));
+  VEDA_TRY(check_ptr(kl_rows, "kl_rows"));
+  VEDA_TRY(check_ptr(kl_out, "kl_out"));
+  if (qtile_rows) VEDA_TRY(check_ptr(qtile_rows, "qtile_rows"));
+  if (!heads_sel || n_heads_sel < 1 || n_heads_sel > VEDA_MAX_HEADS)
+    return fail(VEDA_ERR_INVALID_ARG, "heads_sel must list 1..%d heads", VEDA_MAX_HEADS);
+  if (n_rows < 1) return fail(VEDA_ERR_INVALID_ARG, "n_rows=%d must be >= 1", n_rows);
+  for (int s = 0; s < n_heads_sel; ++s) {
+    if (heads_sel[s] < 0 || heads_sel[s] >= g.heads)
+      return fail(VEDA_ERR_INVALID_ARG, "heads_sel[%d]=%d outside [0, %d)", s, heads_sel[s], g.heads);
+    if (!qtile_rows && n_rows > g.h[heads_sel[s]].nt)
+      return fail(VEDA_ERR_INVALID_ARG, "n_rows=%d exceeds the %d tiles of head %d", n_rows,
+                  g.h[heads_sel[s]].nt, heads_sel[s]);
+  }
+  return after_launch(veda::launch_tilemap_kl(g, heads_sel, n_heads_sel, qtile_rows, n_rows, tilemap, scores,
+                                              kl_rows, kl_out, stream),
+                      "veda_tilemap_kl");
+}
+
 size_t veda_estimator_grad_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows, int32_t hidden,
                                     int32_t out_dim) {
   veda::LayerGeom g;

@@ -517,4 +517,27 @@ cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, c
   return cudaGetLastError();
 }
 
+// The row-wise KL of a finished map (kl_rows_kernel + kl_mean_kernel), for
+// callers that build the map before the scores exist.
+cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int n_heads_sel, const int32_t* rows,
+                              int n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,
+                              cudaStream_t s) {
+  MapParams prm;
+  prm.mode = 0;
+  prm.n_split = 1;
+  prm.ws = nullptr;
+  prm.scale_log2 = 0.f;
+  prm.n_rows = n_rows;
+  prm.rows = rows;
+  prm.tilemap = const_cast<float*>(tilemap);
+  prm.lse = nullptr;
+  for (int i = 0; i < VEDA_MAX_HEADS; ++i) prm.heads_sel[i] = i < n_heads_sel ? heads_sel[i] : 0;
+  const int warps = n_heads_sel * n_rows;
+  kl_rows_kernel<<<(warps * 32 + 255) / 256, 256, 0, s>>>(g, prm, n_heads_sel, scores, kl_rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  kl_mean_kernel<<<1, 1024, 0, s>>>(kl_rows, n_heads_sel, n_rows, kl_out);
+  return cudaGetLastError();
+}
+
 }  // namespace veda

@@ -399,6 +399,9 @@ cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int3
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, int k_cap, float scale, void* op, float* lse,
                                cudaStream_t s);
+cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int n_heads_sel, const int32_t* rows,
+                              int n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,
+                              cudaStream_t s);
 size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile);
 cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, const int32_t* heads_sel,
                            int n_heads_sel, const int32_t* rows, int n_rows, float scale, float* tilemap, float* lse,

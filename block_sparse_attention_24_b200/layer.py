@@ -140,11 +140,30 @@ class VedaLayer:
                             self._grad_loss, stream=stream)
         return self._grads, self._grad_loss
 
-    def forward(self, q, k, v, stream=None):
-        self.front(q, k, v, stream)
-        self.attend(stream)
-        self.distill(stream)
-        return self.o
+    def forward(self, q, k, v, stream=None, out: Optional[torch.Tensor] = None, marks=None):
+        """One step of the hot path, in order on one stream. `marks` (optional
+        dict of CUDA events) is recorded at the stage boundaries "start",
+        "front", "attn0", "attn1", "unpermute", "end". (Running the tile map
+        on a second stream beside the rest measured slower: the split map
+        already fills every SM.)"""
+        main = torch.cuda.current_stream(self.device) if stream is None else stream
+
+        def mark(name):
+            if marks is not None and name in marks:
+                marks[name].record(main)
+
+        mark("start")
+        self.front(q, k, v, main)
+        mark("front")
+        mark("attn0")
+        veda_sparse_attn(self.L, self.qp, self.kp, self.vp, self.idx, self.k, self.k_cap, self.attn_scale, self.op,
+                         stream=main)
+        mark("attn1")
+        veda_permute(self.L, self.o if out is None else out, self.op, inverse=True, stream=main)
+        mark("unpermute")
+        self.distill(main)
+        mark("end")
+        return self.o if out is None else out
 
     def dense(self, out: torch.Tensor, stream=None):
         """Same kernel with every tile kept (the library's own dense path)."""
@@ -194,9 +213,7 @@ class HostPipeline:
             if self.d2h_done[s] is not None:
                 comp.wait_event(self.d2h_done[s])             # slot s's output was copied out
             layer = self.layer
-            layer.front(dq, dk, dv)
-            layer.attend(out=self.outputs[s])
-            layer.distill()
+            layer.forward(dq, dk, dv, out=self.outputs[s])
             if host_kl is not None and layer.maps is not None:
                 host_kl.copy_(layer.kl_out, non_blocking=True)
             done = torch.cuda.Event()

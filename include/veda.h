@@ -201,6 +201,15 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp,
                            float* tilemap, float* lse, const float* scores,
                            float* kl_rows, float* kl_out, float* ws, cudaStream_t stream);
 
+/* The row-wise KL of veda_full_attn_tilemax for a map already built (Veda
+ * summary 2.1, Optimization): kl_rows [n_heads_sel, n_rows] and *kl_out, as
+ * that call computes them when given `scores`. Lets a caller build the map on
+ * one stream, concurrently with the score and top-k calls, and take the KL
+ * once both are done. Arguments as in veda_full_attn_tilemax. */
+int veda_tilemap_kl(const veda_layer* L, const int32_t* heads_sel, int32_t n_heads_sel,
+                    const int32_t* qtile_rows, int32_t n_rows, const float* tilemap,
+                    const float* scores, float* kl_rows, float* kl_out, cudaStream_t stream);
+
 /* Estimator training (Veda summary 2.1, Optimization: the head-specific
  * projections are trained with the row-wise KL against the tile map, with
  * stop-gradient on the pooled descriptors; 2.3, Training Efficiency: on
