@@ -100,6 +100,8 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     rc = lib.veda_full_attn_tilemax(L.ref, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1000), sel, 1, None, 1,
                                     ctypes.c_float(0.1), ctypes.c_void_p(0x1000), None, None, None, None, None, None)
     assert rc == V.VEDA_ERR_INVALID_ARG and "heads_sel" in V.veda_last_error()
+    rc = lib.veda_tilemap_kl(L.ref, sel, 1, None, 1, ctypes.c_void_p(0x1000), None, None, None, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "scores" in V.veda_last_error()
     rc = lib.veda_check_status(None, None)
     assert rc == V.VEDA_ERR_INVALID_ARG
 

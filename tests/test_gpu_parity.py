@@ -489,6 +489,11 @@ def test_tilemap_split_key_range(idx, heads, n_rows):
         V.veda_full_attn_tilemax(L, qp, kp, heads, rows_d, n_rows, scale, tm, lse, scores, klr, klo, ws=ws)
         V.veda_check_status(L)
         out[use_ws] = [t.cpu().double().numpy() for t in (tm, lse, klr, klo[:1])]
+        # the KL of the finished map, taken separately, is the same
+        klr2, klo2 = torch.empty_like(klr), torch.empty_like(klo)
+        V.veda_tilemap_kl(L, heads, rows_d, n_rows, tm, scores, klr2, klo2)
+        torch.cuda.synchronize()
+        assert torch.equal(klr2, klr) and torch.equal(klo2[:1], klo[:1])
     for a, b in zip(out[False], out[True]):
         np.testing.assert_allclose(b, a, rtol=1e-5, atol=1e-30)
     gm = out[True][0]
