@@ -346,7 +346,8 @@ size_t veda_estimator_grad_ws_bytes(const veda_layer* L, int32_t n_heads_sel, in
                                     int32_t out_dim) {
   veda::LayerGeom g;
   if (build_geom(L, &g) != VEDA_OK || n_heads_sel < 1 || n_rows < 1 || hidden < 1 || out_dim < 1) return 0;
-  return (size_t)n_heads_sel * veda::estimator_ws_floats_per_head(g.nt_cap, n_rows, hidden, out_dim) * sizeof(float);
+  return (size_t)n_heads_sel * veda::estimator_ws_floats_per_head(g.nt_cap, n_rows, hidden, out_dim, 3 * g.d) *
+         sizeof(float);
 }
 
 int veda_estimator_grad(const veda_layer* L, const float* dq, const float* dk, const float* w1q, const float* b1q,

@@ -19,7 +19,8 @@
 namespace veda {
 namespace {
 
-constexpr int FW_ROWS = 32;  // descriptors per CTA in the forward recompute
+constexpr int FW_ROWS = 8;   // descriptors per CTA in the forward recompute (small: many CTAs, latency-bound loops)
+constexpr int WG_SPLIT = 8;  // row chunks of the weight-gradient GEMMs (fixed-order partial sums)
 
 __device__ __forceinline__ float gelu_f(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 __device__ __forceinline__ float gelu_grad_f(float x) {
@@ -38,6 +39,7 @@ struct GradWs {
   float* dzq; // [n_rows][hidden]
   float* dzk; // [nt_cap][hidden]
   float* kl;  // [n_rows]
+  float* part;  // [2 sides][WG_SPLIT][(3d+1)*hidden + (hidden+1)*out]  weight-gradient partial sums
 };
 
 struct GradArgs {
@@ -73,7 +75,8 @@ __device__ __forceinline__ GradWs head_ws(const GradArgs& a, int nt_cap, int hs)
   w.dyk = p; p += (size_t)nt_cap * a.out_dim;
   w.dzq = p; p += (size_t)a.n_rows * a.hidden;
   w.dzk = p; p += (size_t)nt_cap * a.hidden;
-  w.kl = p;
+  w.kl = p;  p += (size_t)a.n_rows;
+  w.part = p;
   return w;
 }
 
@@ -89,9 +92,9 @@ __device__ __forceinline__ int desc_row(const GradArgs& a, const LayerGeom& g, i
   return i < nt ? i : -1;
 }
 
-// 1. MLP forward keeping the pre-activations: grid (ceil(N/32), heads_sel,
+// 1. MLP forward keeping the pre-activations: grid (ceil(N/FW_ROWS), heads_sel,
 // 2 sides), 128 threads. Thread u of layer 1 owns hidden unit u (and u+128)
-// for the CTA's 32 descriptors held in shared memory; layer 2 likewise per
+// for the CTA's FW_ROWS descriptors held in shared memory; layer 2 likewise per
 // output unit. Rows past the side's count are written as zeros.
 __global__ void __launch_bounds__(128) fwd_save_kernel(const __grid_constant__ LayerGeom g,
                                                        const __grid_constant__ GradArgs a) {
@@ -244,71 +247,142 @@ __global__ void dy_kernel(const __grid_constant__ LayerGeom g, const __grid_cons
 }
 
 // 4. dz = (dy W2^T) * GELU'(z) for every descriptor row of both sides:
-// grid (rows, heads, sides), thread u owns hidden unit u.
-__global__ void dz_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ GradArgs a) {
-  const int i = blockIdx.x, hs = blockIdx.y, side = blockIdx.z;
+// grid (ceil(rows / DZ_ROWS), heads, sides); thread u owns hidden unit u for
+// the CTA's DZ_ROWS rows (their dy in shared memory), so each W2 entry is
+// loaded once per DZ_ROWS rows.
+constexpr int DZ_ROWS = 8;
+
+__global__ void __launch_bounds__(128) dz_kernel(const __grid_constant__ LayerGeom g,
+                                                 const __grid_constant__ GradArgs a) {
+  extern __shared__ float dys[];  // [DZ_ROWS][out_dim]
+  const int i0 = blockIdx.x * DZ_ROWS, hs = blockIdx.y, side = blockIdx.z;
   const int n_out = side == 0 ? a.n_rows : g.nt_cap;
-  if (i >= n_out) return;
+  if (i0 >= n_out) return;
   const GradWs w = head_ws(a, g.nt_cap, hs);
   const int h = a.heads_sel[hs];
   const float* W2 = a.w2[side] + (long long)h * a.hidden * a.out_dim;
-  const float* dy = (side == 0 ? w.dyq : w.dyk) + (long long)i * a.out_dim;
-  const float* Z = (side == 0 ? w.zq : w.zk) + (long long)i * a.hidden;
-  float* dz = (side == 0 ? w.dzq : w.dzk) + (long long)i * a.hidden;
-  const bool valid = desc_row(a, g, side, hs, i) >= 0;
+  const float* dy = side == 0 ? w.dyq : w.dyk;
+  const float* Z = side == 0 ? w.zq : w.zk;
+  float* dz = side == 0 ? w.dzq : w.dzk;
+  for (int t = threadIdx.x; t < DZ_ROWS * a.out_dim; t += blockDim.x) {
+    const int r = t / a.out_dim;
+    dys[t] = i0 + r < n_out ? dy[(long long)i0 * a.out_dim + t] : 0.f;
+  }
+  __syncthreads();
   for (int u = threadIdx.x; u < a.hidden; u += blockDim.x) {
-    float acc = 0.f;
-    for (int o = 0; o < a.out_dim; ++o) acc = fmaf(dy[o], __ldg(W2 + (long long)u * a.out_dim + o), acc);
-    dz[u] = valid ? acc * gelu_grad_f(Z[u]) : 0.f;
+    float acc[DZ_ROWS] = {};
+    for (int o = 0; o < a.out_dim; ++o) {
+      const float wv = __ldg(W2 + (long long)u * a.out_dim + o);
+#pragma unroll
+      for (int r = 0; r < DZ_ROWS; ++r) acc[r] = fmaf(dys[r * a.out_dim + o], wv, acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < DZ_ROWS; ++r) {
+      const int i = i0 + r;
+      if (i >= n_out) break;
+      const bool valid = desc_row(a, g, side, hs, i) >= 0;
+      dz[(long long)i * a.hidden + u] = valid ? acc[r] * gelu_grad_f(Z[(long long)i * a.hidden + u]) : 0.f;
+    }
   }
 }
 
-// 5. Weight gradients of one side of one selected head: one thread per
-// weight, each summing over that side's descriptor rows in order.
-//   index < din*hidden            : dW1[c][u] = sum_i x[i][c] dz[i][u]
-//   next hidden                    : db1[u]    = sum_i dz[i][u]
-//   next hidden*out_dim            : dW2[u][o] = sum_i GELU(z[i][u]) dy[i][o]
-//   next out_dim                   : db2[o]    = sum_i dy[i][o]
-__global__ void wgrad_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ GradArgs a) {
-  const int hs = blockIdx.y, side = blockIdx.z;
+// 5. Weight gradients of one side of one selected head, as tiled GEMMs over
+// the descriptor rows:
+// out[(K+1) x N] = A^T B with A = [x | 1] (layer 1: K = 3d, N = hidden,
+// B = dz) or A = [GELU(z) | 1] (layer 2: K = hidden, N = out_dim, B = dy);
+// the extra row of ones makes the last output row the bias gradient. A CTA
+// computes a 64 x 64 output tile (4 x 4 per thread) and walks the rows in
+// chunks of 16 in order, so results are bit-reproducible.
+constexpr int WG_TILE = 64, WG_CHUNK = 16;
+
+template <int LAYER>
+__global__ void __launch_bounds__(256) wgrad_gemm_kernel(const __grid_constant__ LayerGeom g,
+                                                         const __grid_constant__ GradArgs a) {
+  __shared__ __align__(16) float As[WG_CHUNK][WG_TILE];
+  __shared__ __align__(16) float Bs[WG_CHUNK][WG_TILE];
+  const int chunk = blockIdx.z % WG_SPLIT;
+  const int hs = (blockIdx.z / WG_SPLIT) >> 1, side = (blockIdx.z / WG_SPLIT) & 1;
   const int h = a.heads_sel[hs];
   const int din = 3 * g.d;
-  const long long n1 = (long long)din * a.hidden, n2 = n1 + a.hidden, n3 = n2 + (long long)a.hidden * a.out_dim,
-                  n4 = n3 + a.out_dim;
-  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= n4) return;
+  const int K = LAYER == 1 ? din : a.hidden;
+  const int N = LAYER == 1 ? a.hidden : a.out_dim;
+  const int k0 = blockIdx.x * WG_TILE, n0 = blockIdx.y * WG_TILE;
   const GradWs w = head_ws(a, g.nt_cap, hs);
-  const int n_in = side == 0 ? a.n_rows : g.nt_cap;
+  const int n_rows_side = side == 0 ? a.n_rows : g.nt_cap;
+  // this CTA's rows: chunk `chunk` of WG_SPLIT, in whole WG_CHUNK steps
+  const int steps = (n_rows_side + WG_CHUNK - 1) / WG_CHUNK;
+  const int i_begin = (int)((long long)steps * chunk / WG_SPLIT) * WG_CHUNK;
+  const int n_in = min(n_rows_side, (int)((long long)steps * (chunk + 1) / WG_SPLIT) * WG_CHUNK);
   const float* X = (side == 0 ? a.dq : a.dk) + (long long)h * g.nt_cap * din;
-  const float* dz = side == 0 ? w.dzq : w.dzk;
-  const float* dy = side == 0 ? w.dyq : w.dyk;
   const float* Z = side == 0 ? w.zq : w.zk;
+  const float* Bsrc = LAYER == 1 ? (side == 0 ? w.dzq : w.dzk) : (side == 0 ? w.dyq : w.dyk);
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int i0 = i_begin; i0 < n_in; i0 += WG_CHUNK) {
+    for (int t = threadIdx.x; t < WG_CHUNK * WG_TILE; t += blockDim.x) {
+      const int ii = t / WG_TILE, cc = t % WG_TILE;
+      const int i = i0 + ii, kk = k0 + cc, nn = n0 + cc;
+      const int row = i < n_in ? desc_row(a, g, side, hs, i) : -1;
+      float av = 0.f, bv = 0.f;
+      if (row >= 0) {
+        if (kk < K) av = LAYER == 1 ? X[(long long)row * din + kk] : gelu_f(Z[(long long)i * a.hidden + kk]);
+        else if (kk == K) av = 1.f;
+        if (nn < N) bv = Bsrc[(long long)i * N + nn];
+      }
+      As[ii][cc] = av;
+      Bs[ii][cc] = bv;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int ii = 0; ii < WG_CHUNK; ++ii) {
+      const float4 av = *reinterpret_cast<const float4*>(&As[ii][ty * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Bs[ii][tx * 4]);
+      const float ar[4] = {av.x, av.y, av.z, av.w}, br[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(ar[u], br[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+  // partial sums of this row chunk: [(K+1) x N] block of the side's partials
+  const long long per_chunk = (long long)(din + 1) * a.hidden + (long long)(a.hidden + 1) * a.out_dim;
+  float* P = w.part + ((long long)side * WG_SPLIT + chunk) * per_chunk +
+             (LAYER == 1 ? 0 : (long long)(din + 1) * a.hidden);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int kk = k0 + ty * 4 + u;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int nn = n0 + tx * 4 + v;
+      if (nn < N && kk <= K) P[(long long)kk * N + nn] = acc[u][v];
+    }
+  }
+}
+
+// Sum of the row chunks' partials in chunk order: weight and bias gradients
+// of one side of one selected head (grid: elements, heads x sides).
+__global__ void wgrad_reduce_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ GradArgs a) {
+  const int hs = blockIdx.y >> 1, side = blockIdx.y & 1;
+  const int h = a.heads_sel[hs];
+  const int din = 3 * g.d;
+  const long long n1 = (long long)(din + 1) * a.hidden, per_chunk = n1 + (long long)(a.hidden + 1) * a.out_dim;
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= per_chunk) return;
+  const GradWs w = head_ws(a, g.nt_cap, hs);
+  const float* P = w.part + (long long)side * WG_SPLIT * per_chunk + t;
   float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < WG_SPLIT; ++c) acc += P[c * per_chunk];
   if (t < n1) {
-    const int c = (int)(t / a.hidden), u = (int)(t % a.hidden);
-    for (int i = 0; i < n_in; ++i) {
-      const int row = desc_row(a, g, side, hs, i);
-      if (row >= 0) acc = fmaf(X[(long long)row * din + c], dz[(long long)i * a.hidden + u], acc);
-    }
-    a.gw1[side][(long long)h * n1 + t] = acc;
-  } else if (t < n2) {
-    const int u = (int)(t - n1);
-    for (int i = 0; i < n_in; ++i)
-      if (desc_row(a, g, side, hs, i) >= 0) acc += dz[(long long)i * a.hidden + u];
-    a.gb1[side][(long long)h * a.hidden + u] = acc;
-  } else if (t < n3) {
-    const long long e = t - n2;
-    const int u = (int)(e / a.out_dim), o = (int)(e % a.out_dim);
-    for (int i = 0; i < n_in; ++i) {
-      if (desc_row(a, g, side, hs, i) < 0) continue;
-      acc = fmaf(gelu_f(Z[(long long)i * a.hidden + u]), dy[(long long)i * a.out_dim + o], acc);
-    }
-    a.gw2[side][(long long)h * a.hidden * a.out_dim + e] = acc;
+    const int kk = (int)(t / a.hidden), nn = (int)(t % a.hidden);
+    if (kk < din) a.gw1[side][((long long)h * din + kk) * a.hidden + nn] = acc;
+    else a.gb1[side][(long long)h * a.hidden + nn] = acc;
   } else {
-    const int o = (int)(t - n3);
-    for (int i = 0; i < n_in; ++i)
-      if (desc_row(a, g, side, hs, i) >= 0) acc += dy[(long long)i * a.out_dim + o];
-    a.gb2[side][(long long)h * a.out_dim + o] = acc;
+    const long long e = t - n1;
+    const int kk = (int)(e / a.out_dim), nn = (int)(e % a.out_dim);
+    if (kk < a.hidden) a.gw2[side][((long long)h * a.hidden + kk) * a.out_dim + nn] = acc;
+    else a.gb2[side][(long long)h * a.out_dim + nn] = acc;
   }
 }
 
@@ -327,9 +401,10 @@ __global__ void loss_kernel(const __grid_constant__ LayerGeom g, const __grid_co
 
 }  // namespace
 
-size_t estimator_ws_floats_per_head(int nt_cap, int n_rows, int hidden, int out_dim) {
+size_t estimator_ws_floats_per_head(int nt_cap, int n_rows, int hidden, int out_dim, int din) {
   return 2 * (size_t)n_rows * hidden + 2 * (size_t)n_rows * out_dim + 2 * (size_t)nt_cap * hidden +
-         2 * (size_t)nt_cap * out_dim + (size_t)n_rows * nt_cap + (size_t)n_rows;
+         2 * (size_t)nt_cap * out_dim + (size_t)n_rows * nt_cap + (size_t)n_rows +
+         2 * (size_t)WG_SPLIT * ((size_t)(din + 1) * hidden + (size_t)(hidden + 1) * out_dim);
 }
 
 cudaError_t launch_estimator_grad(const LayerGeom& g, const float* dq, const float* dk, const float* const w[8],
@@ -359,7 +434,7 @@ cudaError_t launch_estimator_grad(const LayerGeom& g, const float* dq, const flo
   a.scale = scale;
   a.coef = 1.0f / ((float)n_rows * (float)n_heads_sel);
   for (int i = 0; i < n_heads_sel; ++i) a.heads_sel[i] = heads_sel[i];
-  a.ws_per_head = estimator_ws_floats_per_head(g.nt_cap, n_rows, hidden, out_dim);
+  a.ws_per_head = estimator_ws_floats_per_head(g.nt_cap, n_rows, hidden, out_dim, 3 * g.d);
   a.ws = ws;
   const int din = 3 * g.d;
   // gradients of heads that are not selected are zero
@@ -379,9 +454,16 @@ cudaError_t launch_estimator_grad(const LayerGeom& g, const float* dq, const flo
   if (e != cudaSuccess) return e;
   kl_grad_kernel<<<dim3(n_rows, n_heads_sel), 256, smem_kl, s>>>(g, a);
   dy_kernel<<<dim3(n_side_max, n_heads_sel, 2), 128, 0, s>>>(g, a);
-  dz_kernel<<<dim3(n_side_max, n_heads_sel, 2), 128, 0, s>>>(g, a);
-  const long long nw = (long long)n1 + n2 + n3 + n4;
-  wgrad_kernel<<<dim3((unsigned)((nw + 255) / 256), n_heads_sel, 2), 256, 0, s>>>(g, a);
+  dz_kernel<<<dim3((n_side_max + DZ_ROWS - 1) / DZ_ROWS, n_heads_sel, 2), 128,
+              (size_t)DZ_ROWS * out_dim * sizeof(float), s>>>(g, a);
+  wgrad_gemm_kernel<1><<<dim3((din + 1 + WG_TILE - 1) / WG_TILE, (hidden + WG_TILE - 1) / WG_TILE,
+                              2 * n_heads_sel * WG_SPLIT),
+                         256, 0, s>>>(g, a);
+  wgrad_gemm_kernel<2><<<dim3((hidden + 1 + WG_TILE - 1) / WG_TILE, (out_dim + WG_TILE - 1) / WG_TILE,
+                              2 * n_heads_sel * WG_SPLIT),
+                         256, 0, s>>>(g, a);
+  const long long per_chunk = (long long)(din + 1) * hidden + (long long)(hidden + 1) * out_dim;
+  wgrad_reduce_kernel<<<dim3((unsigned)((per_chunk + 255) / 256), 2 * n_heads_sel), 256, 0, s>>>(g, a);
   loss_kernel<<<1, 32, 0, s>>>(g, a);
   return cudaGetLastError();
 }

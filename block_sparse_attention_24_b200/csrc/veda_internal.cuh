@@ -384,7 +384,7 @@ cudaError_t launch_mlp(const LayerGeom& g, const float* dq, const float* dk, con
                        const float* b2k, int hidden, int out_dim, float* emb_ws, cudaStream_t s);
 cudaError_t launch_score_topk(const LayerGeom& g, const float* emb_ws, int out_dim, float scale, int k_cap,
                               int32_t* idx, uint8_t* mask, float* scores, cudaStream_t s);
-size_t estimator_ws_floats_per_head(int nt_cap, int n_rows, int hidden, int out_dim);
+size_t estimator_ws_floats_per_head(int nt_cap, int n_rows, int hidden, int out_dim, int din);
 cudaError_t launch_estimator_grad(const LayerGeom& g, const float* dq, const float* dk, const float* const w[8],
                                   float* const gw[8], int hidden, int out_dim, float scale, const int32_t* heads_sel,
                                   int n_heads_sel, const int32_t* rows, int n_rows, const float* tilemap,
