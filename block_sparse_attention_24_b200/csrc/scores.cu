@@ -13,17 +13,18 @@
 namespace veda {
 namespace {
 
-constexpr int MLP_ROWS = 32;
+constexpr int MLP_ROWS = 32;         // descriptors per CTA (16 measured no faster)
+constexpr int MLP_RPT = MLP_ROWS / 4;  // rows per thread (4 warps, one row group each)
 
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
-// grid (ceil(nt_cap/32), heads, B*2): z%2 == 0 -> query side, 1 -> key side.
-// 32 tile descriptors per CTA, kept transposed in shared memory (input-major)
-// so that a thread's 8 rows are two 16-byte loads. Each of the 128 threads
-// owns an 8-row x 4-column register tile of the current layer (32 fp32
-// accumulators, 32 FMAs per 16-byte weight load); layer 1 is applied in
-// chunks of 128 hidden units, GELU'd and transposed into shared memory for
-// layer 2.
+// grid (ceil(nt_cap/MLP_ROWS), heads, B*2): z%2 == 0 -> query side, 1 -> key
+// side. MLP_ROWS tile descriptors per CTA, kept transposed in shared memory
+// (input-major) so that a thread's rows are 16-byte loads. Each of the 128
+// threads owns an MLP_RPT-row x 4-column register tile of the current layer
+// (4*MLP_RPT FMAs per 16-byte weight load); layer 1 is applied in chunks of
+// 128 hidden units, GELU'd and transposed into shared memory for layer 2.
+// (Half the rows per CTA, for more resident CTAs, measured no faster.)
 __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerGeom g, const float* __restrict__ dq,
                                                   const float* __restrict__ dk, const float* __restrict__ w1q,
                                                   const float* __restrict__ b1q, const float* __restrict__ w2q,
@@ -59,17 +60,17 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
     xsT[(4 * c4 + 3) * MLP_ROWS + r] = v.w;
   }
   __syncthreads();
-  const int rg = threadIdx.x / 32;  // rows rg*8 .. rg*8+7 (one warp per row group)
+  const int rg = threadIdx.x / 32;  // rows rg*MLP_RPT .. (one warp per row group)
   const int cg = threadIdx.x % 32;  // columns cg*4 .. cg*4+3 of a 128-column chunk
 
   // layer 1 + GELU
   for (int cb = 0; cb < hidden; cb += 128) {
     const int c = cb + cg * 4;
     if (c < hidden) {
-      float acc[8][4];
+      float acc[MLP_RPT][4];
       const float4 bias = __ldg(reinterpret_cast<const float4*>(B1 + c));
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
+      for (int r = 0; r < MLP_RPT; ++r) {
         acc[r][0] = bias.x;
         acc[r][1] = bias.y;
         acc[r][2] = bias.z;
@@ -78,23 +79,29 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
 #pragma unroll 4
       for (int i = 0; i < din; ++i) {
         const float4 wv = __ldg(reinterpret_cast<const float4*>(W1 + (long long)i * hidden + c));
-        const float4 x0 = *reinterpret_cast<const float4*>(xsT + i * MLP_ROWS + rg * 8);
-        const float4 x1 = *reinterpret_cast<const float4*>(xsT + i * MLP_ROWS + rg * 8 + 4);
-        const float xr[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        float xr[MLP_RPT];
+#pragma unroll
+        for (int q = 0; q < MLP_RPT / 4; ++q) {
+          const float4 x4 = *reinterpret_cast<const float4*>(xsT + i * MLP_ROWS + rg * MLP_RPT + 4 * q);
+          xr[4 * q] = x4.x; xr[4 * q + 1] = x4.y; xr[4 * q + 2] = x4.z; xr[4 * q + 3] = x4.w;
+        }
         const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int r = 0; r < MLP_RPT; ++r)
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(xr[r], wr[e], acc[r][e]);
       }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float4 v0, v1;
-        v0.x = gelu_erf(acc[0][e]); v0.y = gelu_erf(acc[1][e]); v0.z = gelu_erf(acc[2][e]); v0.w = gelu_erf(acc[3][e]);
-        v1.x = gelu_erf(acc[4][e]); v1.y = gelu_erf(acc[5][e]); v1.z = gelu_erf(acc[6][e]); v1.w = gelu_erf(acc[7][e]);
-        *reinterpret_cast<float4*>(hsT + (c + e) * MLP_ROWS + rg * 8) = v0;
-        *reinterpret_cast<float4*>(hsT + (c + e) * MLP_ROWS + rg * 8 + 4) = v1;
-      }
+      for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int q = 0; q < MLP_RPT / 4; ++q) {
+          float4 v;
+          v.x = gelu_erf(acc[4 * q][e]);
+          v.y = gelu_erf(acc[4 * q + 1][e]);
+          v.z = gelu_erf(acc[4 * q + 2][e]);
+          v.w = gelu_erf(acc[4 * q + 3][e]);
+          *reinterpret_cast<float4*>(hsT + (c + e) * MLP_ROWS + rg * MLP_RPT + 4 * q) = v;
+        }
     }
   }
   __syncthreads();
@@ -102,10 +109,10 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
   for (int cb = 0; cb < out_dim; cb += 128) {
     const int c = cb + cg * 4;
     if (c >= out_dim) continue;
-    float acc[8][4];
+    float acc[MLP_RPT][4];
     const float4 bias = __ldg(reinterpret_cast<const float4*>(B2 + c));
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
+    for (int r = 0; r < MLP_RPT; ++r) {
       acc[r][0] = bias.x;
       acc[r][1] = bias.y;
       acc[r][2] = bias.z;
@@ -114,18 +121,21 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
 #pragma unroll 4
     for (int i = 0; i < hidden; ++i) {
       const float4 wv = __ldg(reinterpret_cast<const float4*>(W2 + (long long)i * out_dim + c));
-      const float4 x0 = *reinterpret_cast<const float4*>(hsT + i * MLP_ROWS + rg * 8);
-      const float4 x1 = *reinterpret_cast<const float4*>(hsT + i * MLP_ROWS + rg * 8 + 4);
-      const float xr[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      float xr[MLP_RPT];
+#pragma unroll
+      for (int q = 0; q < MLP_RPT / 4; ++q) {
+        const float4 x4 = *reinterpret_cast<const float4*>(hsT + i * MLP_ROWS + rg * MLP_RPT + 4 * q);
+        xr[4 * q] = x4.x; xr[4 * q + 1] = x4.y; xr[4 * q + 2] = x4.z; xr[4 * q + 3] = x4.w;
+      }
       const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+      for (int r = 0; r < MLP_RPT; ++r)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(xr[r], wr[e], acc[r][e]);
     }
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int row = r0 + rg * 8 + r;
+    for (int r = 0; r < MLP_RPT; ++r) {
+      const int row = r0 + rg * MLP_RPT + r;
       if (row < g.nt_cap) {
         const bool v = row < nt;
         *reinterpret_cast<float4*>(out + (long long)row * out_dim + c) =
