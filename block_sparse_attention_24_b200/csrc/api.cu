@@ -278,7 +278,7 @@ int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const 
 size_t veda_full_attn_tilemax_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows) {
   veda::LayerGeom g;
   if (build_geom(L, &g) != VEDA_OK || n_heads_sel < 1 || n_rows < 1) return 0;
-  return veda::tilemax_ws_bytes(n_heads_sel, n_rows, g.tile);
+  return veda::tilemax_ws_bytes(n_heads_sel, n_rows, g.tile, g.nt_cap);
 }
 
 int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp, const int32_t* heads_sel,

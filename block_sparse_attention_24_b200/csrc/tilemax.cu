@@ -3,13 +3,20 @@
 // passes, on a subset of query tiles).
 //
 // Two 128-row blocks of selected query tiles share one CTA and every K block
-// load; each sweeps all key blocks twice with tcgen05 S = Q K^T:
+// load. M[a, b] = max over the tile region of the softmax probability =
+// exp2(max over the tile's valid rows of (row's largest logit in key tile b
+// * C - row's log2-sum-exp)). Without a workspace each CTA sweeps all key
+// blocks twice with tcgen05 S = Q K^T:
 //   pass 1: per row, log2-domain log-sum-exp over all valid keys;
 //   pass 2: per row and key tile, the largest logit minus lse, then the
 //           maximum over the tile's valid rows (warp shuffle, then a shared
-//           order-preserving atomicMax) -> M[a, b] = exp2(.) = max-pooled
-//           softmax probability over the tile region.
-// A second kernel turns map rows and score rows into KL values, a third
+//           order-preserving atomicMax).
+// With a workspace the key range may be split over several CTAs and there is
+// one sweep: it writes each row's partial (reference, sum) and its largest
+// logit per key tile; map_finish_kernel combines the partial sums in a fixed
+// order and reduces the stored maxima over rows (the same values pass 2 would
+// recompute, so the same map).
+// A further kernel turns map rows and score rows into KL values, another
 // averages them in a fixed order.
 #include <climits>
 
@@ -45,9 +52,10 @@ struct MapLayout {
 
 struct MapParams {
   float scale_log2;
-  int mode;             // 0: both passes; 1: pass 1 only, partial sums to ws; 2: pass 2 only, from ws
+  int mode;             // 0: both passes; 1: one sweep, partial sums and row maxima to ws
   int n_split;          // CTAs sharing one row pair's key range (blockIdx.z); 1 for mode 0
   float2* ws;           // [n_heads_sel][n_rows][tile][n_split] (reference m, sum l) in log2 units
+  float* rowmax;        // [n_heads_sel][n_rows][nt_cap][tile] largest logit per row and key tile
   int n_rows;
   const int32_t* rows;  // [n_heads_sel, n_rows] or NULL
   float* tilemap;       // [n_heads_sel, n_rows, nt_cap]
@@ -110,9 +118,10 @@ __device__ __forceinline__ float tile_expsum(const uint32_t (&u)[BN], int c0, in
 
 // One CTA owns two 128-row blocks (A, B) of selected query rows of one head:
 // one 128-token query tile each, or two 64-token query tiles each. Both
-// sweep every key block twice (pass 1: log-sum-exp; pass 2: per key tile
-// max of logit - lse, then max over the tile's rows); each K block is loaded
-// once for both. S of each row block is double-buffered in TMEM, so the MMA
+// sweep every key block of the CTA's range, twice in mode 0 (pass 1:
+// log-sum-exp; pass 2: per key tile max of logit - lse, then max over the
+// tile's rows), once in mode 1 (partial log-sum-exp and per key tile row
+// maxima to the workspace); each K block is loaded once for both. S of each row block is double-buffered in TMEM, so the MMA
 // for the next key block overlaps the softmax of the current one.
 //   warps 0-3 / 4-7  row block A / B (thread = row = TMEM lane)
 //   warp 8           TMA producer (Q once, then K blocks, 3-stage ring)
@@ -272,20 +281,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto part_ws = [&](int sp) -> float2* {
       return prm.ws + (((long long)hs * prm.n_rows + e_row) * TILE + (row % TILE)) * prm.n_split + sp;
     };
-    if (prm.mode == 2 && rb_valid[r] && e_row < prm.n_rows) {
-      // combine the splits' partial sums in a fixed order: every split's CTA
-      // gets the same log-sum-exp
-      float M = -INFINITY;
-      for (int sp = 0; sp < prm.n_split; ++sp) M = fmaxf(M, part_ws(sp)->x);
-      float L = 0.f;
-      for (int sp = 0; sp < prm.n_split; ++sp) {
-        const float2 pr = *part_ws(sp);
-        if (pr.y > 0.f) L += pr.y * fast_exp2(pr.x - M);
-      }
-      lse2 = M + __log2f(L);
-      if (prm.lse && split == 0)
-        prm.lse[((long long)hs * prm.n_rows + e_row) * TILE + (row % TILE)] = row_valid ? lse2 * 0.69314718055994531f : 0.f;
-    }
+    const bool keep_max = prm.mode == 1 && e_row < prm.n_rows;
     for (int it = 0; it < (rb_valid[r] ? iters : 0); ++it) {
       const int sb = 2 * r + (it & 1);
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, (it >> 1) & 1, abort_flag, g.dev_status))) break;
@@ -295,7 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       mbar_arrive(s_free + sb);  // S buffer may be overwritten now
       const int kb = kb_begin + it % nkb;
-      const bool pass2 = prm.mode == 2 || (prm.mode == 0 && it >= nkb);
+      const bool pass2 = prm.mode == 0 && it >= nkb;
 #pragma unroll
       for (int uu = 0; uu < NSUB; ++uu) {
         const int kt = kb * NSUB + uu;
@@ -315,10 +311,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // relative precision, and move it only when a tile's sum nears the
           // top of the range (rare).
           if (klen > 0) {
-            if (m == -INFINITY) m = block_max() * C;
+            float mx = 0.f;
+            if (keep_max) {  // the row's largest logit in key tile kt, for the map
+              mx = block_max();
+              prm.rowmax[(((long long)hs * prm.n_rows + e_row) * g.nt_cap + kt) * TILE + (row % TILE)] = mx;
+            }
+            if (m == -INFINITY) m = (keep_max ? mx : block_max()) * C;
             float sum = block_sum(m);
             if (!(sum <= OVERFLOW_SUM)) {
-              const float mnew = fmaxf(m, block_max() * C);
+              const float mnew = fmaxf(m, (keep_max ? mx : block_max()) * C);
               l *= fast_exp2(m - mnew);
               m = mnew;
               sum = block_sum(m);
@@ -347,11 +348,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
-  // write the map rows: this CTA's key tiles (the last split also writes
-  // the zero columns past nt)
-  const int kt_begin = kb_begin * NSUB;
-  const int kt_end = split == prm.n_split - 1 ? g.nt_cap : kb_end * NSUB;
-  if (!*abort_flag && prm.mode != 1) {
+  // mode 0: write the map rows (zero columns past nt included)
+  const int kt_begin = 0, kt_end = g.nt_cap;
+  if (!*abort_flag && prm.mode == 0) {
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -364,6 +363,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           out[b] = (b < nt && k != 0u && qv[r][s]) ? fast_exp2(unord_f32(k)) : 0.f;
         }
       }
+  }
+}
+
+constexpr int FIN_THREADS = 256;
+constexpr int FIN_KT = 64;  // key tiles per finishing CTA
+
+// Finishes a mode-1 map: per row, the fixed-order combination of the splits'
+// partial (reference, sum) into the log2-sum-exp; per key tile, the maximum
+// over the query tile's valid rows of (largest logit * C - lse), as 2^max.
+// Grid: (key-tile chunks, selected rows, selected heads); warp per key tile.
+template <int TILE>
+__global__ void __launch_bounds__(FIN_THREADS)
+    map_finish_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ MapParams prm) {
+  __shared__ float lse2s[TILE];
+  const int hs = blockIdx.z;
+  const int h = prm.heads_sel[hs];
+  const HeadGeom& hg = g.h[h];
+  const int nt = hg.nt;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const float C = prm.scale_log2;
+  const int kt_end = min(g.nt_cap, (int)(blockIdx.x + 1) * FIN_KT);
+  for (int e = blockIdx.y; e < prm.n_rows; e += gridDim.y) {
+    const int a = prm.rows ? __ldg(prm.rows + (long long)hs * prm.n_rows + e) : e;
+    const bool qv = a >= 0 && a < nt;  // a bad entry was reported by the sweep
+    const int len = qv ? tile_len(hg, g.T, a) : 0;
+    const long long er = (long long)hs * prm.n_rows + e;
+    __syncthreads();  // lse2s of the previous row is no longer read
+    if (threadIdx.x < TILE) {
+      const int row = threadIdx.x;
+      const float2* part = prm.ws + (er * TILE + row) * prm.n_split;
+      float M = -INFINITY;
+      for (int sp = 0; sp < prm.n_split; ++sp) M = fmaxf(M, part[sp].x);
+      float L = 0.f;
+      for (int sp = 0; sp < prm.n_split; ++sp) {
+        const float2 pr = part[sp];
+        if (pr.y > 0.f) L += pr.y * fast_exp2(pr.x - M);
+      }
+      const float lse2 = M + __log2f(L);
+      lse2s[row] = lse2;
+      if (prm.lse && blockIdx.x == 0) prm.lse[er * TILE + row] = row < len ? lse2 * 0.69314718055994531f : 0.f;
+    }
+    __syncthreads();
+    for (int kt = blockIdx.x * FIN_KT + warp; kt < kt_end; kt += FIN_THREADS / 32) {
+      float out = 0.f;
+      if (kt < nt && qv) {
+        const float* mx = prm.rowmax + (er * g.nt_cap + kt) * TILE;
+        float v = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < TILE / 32; ++j) {
+          const int row = lane + 32 * j;
+          if (row < len) v = fmaxf(v, fmaf(__ldg(mx + row), C, -lse2s[row]));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+        out = v > -INFINITY ? fast_exp2(v) : 0.f;
+      }
+      if (lane == 0) prm.tilemap[er * g.nt_cap + kt] = out;
+    }
   }
 }
 
@@ -443,9 +500,9 @@ cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, Map
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int pairs = (prm.n_rows + 2 * NSUB - 1) / (2 * NSUB);
-  // With a workspace, split each row pair's key range over n_split CTAs when
-  // that fills the SMs' waves noticeably better (one CTA per SM): pass 1
-  // writes partial sums, pass 2 combines them and builds its own key tiles.
+  // With a workspace: one sweep (mode 1), with each row pair's key range split
+  // over n_split CTAs when that fills the SMs' waves noticeably better (one
+  // CTA per SM), then map_finish_kernel.
   int n_split = 1;
   if (prm.ws) {
     int dev = 0, sms = 148;
@@ -468,7 +525,7 @@ cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, Map
         n_split = sp;
       }
   }
-  if (n_split == 1) {
+  if (!prm.ws) {
     prm.mode = 0;
     prm.n_split = 1;
     kern<<<dim3(pairs, n_heads_sel, 1), NUM_THREADS, smem, s>>>(g, tq, tk, prm);
@@ -479,15 +536,18 @@ cudaError_t launch_map_t(const LayerGeom& g, const void* qp, const void* kp, Map
   kern<<<dim3(pairs, n_heads_sel, n_split), NUM_THREADS, smem, s>>>(g, tq, tk, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  prm.mode = 2;
-  kern<<<dim3(pairs, n_heads_sel, n_split), NUM_THREADS, smem, s>>>(g, tq, tk, prm);
+  const dim3 fgrid((g.nt_cap + FIN_KT - 1) / FIN_KT, prm.n_rows < 65535 ? prm.n_rows : 65535, n_heads_sel);
+  map_finish_kernel<TILE><<<fgrid, FIN_THREADS, 0, s>>>(g, prm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile) {
-  return (size_t)n_heads_sel * n_rows * tile * MAP_MAX_SPLIT * sizeof(float2);
+// partial sums [heads][rows][tile][MAP_MAX_SPLIT] float2, then the row
+// maxima [heads][rows][nt_cap][tile] float
+size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile, int nt_cap) {
+  const size_t rows = (size_t)n_heads_sel * n_rows * tile;
+  return rows * MAP_MAX_SPLIT * sizeof(float2) + rows * nt_cap * sizeof(float);
 }
 
 cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, const int32_t* heads_sel,
@@ -497,6 +557,7 @@ cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, c
   prm.mode = 0;
   prm.n_split = 1;
   prm.ws = reinterpret_cast<float2*>(ws);
+  prm.rowmax = ws ? ws + (size_t)n_heads_sel * n_rows * g.tile * MAP_MAX_SPLIT * 2 : nullptr;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.n_rows = n_rows;
   prm.rows = rows;
@@ -526,6 +587,7 @@ cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int 
   prm.mode = 0;
   prm.n_split = 1;
   prm.ws = nullptr;
+  prm.rowmax = nullptr;
   prm.scale_log2 = 0.f;
   prm.n_rows = n_rows;
   prm.rows = rows;

@@ -402,7 +402,7 @@ cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* k
 cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int n_heads_sel, const int32_t* rows,
                               int n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,
                               cudaStream_t s);
-size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile);
+size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile, int nt_cap);
 cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, const int32_t* heads_sel,
                            int n_heads_sel, const int32_t* rows, int n_rows, float scale, float* tilemap, float* lse,
                            const float* scores, float* kl_rows, float* kl_out, float* ws, cudaStream_t s);

@@ -190,10 +190,14 @@ int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const 
  * receives KL(t || softmax(scores row)) with t the tile-map row normalised to
  * sum 1, and *kl_out (device fp32) their mean over rows, then heads.
  * ws (may be NULL): veda_full_attn_tilemax_ws_bytes(...) bytes of device
- * scratch; with it the call may split each pair of query tiles' key range
- * over several CTAs (two launches: partial sums, then their fixed-order
- * combination) so that small maps fill every SM; results are the same up to
- * fp32 rounding of the log-sum-exp. Only B == 1 layers are accepted. */
+ * scratch (partial sums, and every selected row's largest logit per key tile:
+ * 4 * n_heads_sel * n_rows * tile * nt_cap bytes of it). With it the logits
+ * are computed once instead of twice: one sweep, whose key range may be
+ * split over several CTAs so that small maps fill every SM, stores partial
+ * sums and row maxima; a second kernel combines the sums in a fixed order and
+ * reduces the maxima. Without it each CTA sweeps its keys twice. Results are
+ * the same up to fp32 rounding of the log-sum-exp. Only B == 1 layers are
+ * accepted. */
 size_t veda_full_attn_tilemax_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows);
 int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp,
                            const int32_t* heads_sel, int32_t n_heads_sel,
