@@ -30,6 +30,7 @@
 // Every mbarrier wait is bounded (VEDA_WAIT_LIMIT_NS); on expiry the CTA
 // records VEDA_ERR_TIMEOUT, drains what it issued, frees its TMEM and exits.
 #include <climits>
+#include <type_traits>
 
 #include "veda_internal.cuh"
 
@@ -39,6 +40,7 @@ namespace {
 constexpr int BM = 128;               // rows per query tile
 constexpr int BN = 128;               // keys per tile
 constexpr int KST = 2, VST = 3;       // K and V ring stages
+constexpr int SDR = 4;                // step-done barriers (ring over union positions)
 constexpr float OVERFLOW_SUM = 1.8446744e19f;  // 2^64: a tile's P sum above this moves the reference
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_THREADS = 384;
@@ -55,8 +57,8 @@ struct PairLayout {
   static constexpr int OFF_K = 2 * QB;
   static constexpr int OFF_V = OFF_K + KST * KB;
   static constexpr int OFF_BAR = OFF_V + VST * KB;
-  // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1;
+  // q_full, k_full[KST], v_full[VST], step_done[SDR], s_full[2], p_full[2], pv_done[2], drain
+  static constexpr int NUM_BARS = 1 + KST + VST + SDR + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
@@ -84,25 +86,44 @@ __device__ __forceinline__ int list_tile(const int32_t* row, int j, int nt, int3
 
 // Walks the merge of two kept-tile lists: each call yields the next tile and
 // which of the two query tiles kept it. Every entry of both lists is visited
-// exactly once; equal entries are merged.
+// exactly once; equal entries are merged. Each list's entry after the current
+// one is loaded one step ahead and range-checked only when it becomes current,
+// so a call never waits for a load.
 struct UnionWalk {
   const int32_t* la;
   const int32_t* lb;
   int ka, kb, ia, ib, nt;
-  int ta, tb;
+  int ta, tb;          // current entries (range-checked), INT_MAX past the end
+  int ra, rb;          // raw next entries
   int32_t* status;
+  __device__ int raw(const int32_t* l, int j, int k) { return j < k ? (l ? __ldg(l + j) : j) : 0; }
+  __device__ int checked(int t, bool report_bad) {
+    if (t < 0 || t >= nt) {
+      if (report_bad && status) report(status, VEDA_ERR_BAD_INDEX);
+      t = 0;
+    }
+    return t;
+  }
   __device__ UnionWalk(const int32_t* a, int na, const int32_t* b, int nb, int nt_, int32_t* st)
       : la(a), lb(b), ka(na), kb(nb), ia(0), ib(0), nt(nt_), status(st) {
-    ta = ka > 0 ? list_tile(la, 0, nt, status) : INT_MAX;
-    tb = kb > 0 ? list_tile(lb, 0, nt, nullptr) : INT_MAX;
+    ta = ka > 0 ? checked(raw(la, 0, ka), true) : INT_MAX;
+    tb = kb > 0 ? checked(raw(lb, 0, kb), true) : INT_MAX;
+    ra = raw(la, 1, ka);
+    rb = raw(lb, 1, kb);
   }
   __device__ bool next(int& t, bool& ma, bool& mb) {
     if (ia >= ka && ib >= kb) return false;
     t = ta < tb ? ta : tb;
     ma = ta == t;
     mb = tb == t;
-    if (ma) ta = ++ia < ka ? list_tile(la, ia, nt, status) : INT_MAX;
-    if (mb) tb = ++ib < kb ? list_tile(lb, ib, nt, nullptr) : INT_MAX;
+    if (ma) {
+      ta = ++ia < ka ? checked(ra, true) : INT_MAX;
+      ra = raw(la, ia + 1, ka);
+    }
+    if (mb) {
+      tb = ++ib < kb ? checked(rb, true) : INT_MAX;
+      rb = raw(lb, ib + 1, kb);
+    }
     return true;
   }
 };
@@ -212,12 +233,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + KST;
-  uint64_t* v_full = k_empty + KST;
-  uint64_t* v_empty = v_full + VST;
-  uint64_t* s_full = v_empty + VST;  // [2]
+  uint64_t* v_full = k_full + KST;
+  uint64_t* step_done = v_full + VST;  // [SDR]: all MMAs of union position e issued, and P V of e-1
+  uint64_t* s_full = step_done + SDR;  // [2]
   uint64_t* p_full = s_full + 2;     // [2], 128 arrivals each
-  uint64_t* pv_done = p_full + 2;    // [2]
+  uint64_t* pv_done = p_full + 2;    // [2], one phase: the query tile's last P V
   uint64_t* mma_drain = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
@@ -245,7 +265,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool is_k = warp == 8;
       const CUtensorMap* map = is_k ? &tmK : &tmV;
       uint64_t* full = is_k ? k_full : v_full;
-      uint64_t* empty = is_k ? k_empty : v_empty;
       const int ST = is_k ? KST : VST;
       uint8_t* ring = smem + (is_k ? Lay::OFF_K : Lay::OFF_V);
       tma_prefetch_desc(map);
@@ -263,7 +282,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ma, mb;
       while (uw.next(t, ma, mb)) {
         const int st = e % ST;
-        if (e >= ST && !mbar_wait(empty + st, ((e - ST) / ST) & 1, abort_flag, g.dev_status)) break;
+        // slot reuse: K of position e-KST is free once its S MMAs completed
+        // (step e-KST); V of e-VST once its P V completed (issued by the end
+        // of step e-VST+1)
+        const int sd = e - ST + (is_k ? 0 : 1);
+        if (e >= ST && !mbar_wait(step_done + sd % SDR, (sd / SDR) & 1, abort_flag, g.dev_status)) break;
         mbar_expect_tx(full + st, Lay::KB);
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
@@ -287,15 +310,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t dQ = sdesc_sw128(smem_u32(smem + Lay::OFF_Q), 16, 1024);
       const uint64_t dK = sdesc_sw128(smem_u32(smem + Lay::OFF_K), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(smem + Lay::OFF_V), BN * 128, 1024);
-      bool pend[2] = {false, false};
-      int js[2] = {0, 0};  // S issued per query tile
+      // Per query tile state in scalars, and P V / S issue specialised per
+      // query tile at compile time: this thread's bookkeeping between MMA
+      // batches is on the critical path, and nothing here may live in local
+      // memory.
+      bool pend0 = false, pend1 = false;  // a P V is pending
+      int js0 = 0, js1 = 0;               // S issued
       int prev_e = -1;
       bool ok = mbar_wait(q_full, 0, abort_flag, g.dev_status);
       if (ok) tc_fence_after();
-      // P V for the tile kept at union position prev_e by query tile r
-      auto issue_pv = [&](int r) -> bool {
+      using I0 = std::integral_constant<int, 0>;
+      using I1 = std::integral_constant<int, 1>;
+      // P V for the tile query tile r kept at union position prev_e
+      auto issue_pv = [&](auto rc) -> bool {
+        constexpr int r = decltype(rc)::value;
+        int& js = r ? js1 : js0;
+        bool& pend = r ? pend1 : pend0;
         const int vs = prev_e % VST;
-        if (!mbar_wait(p_full + r, (js[r] - 1) & 1, abort_flag, g.dev_status)) return false;
+        if (!mbar_wait(p_full + r, (js - 1) & 1, abort_flag, g.dev_status)) return false;
         if (!mbar_wait(v_full + vs, (prev_e / VST) & 1, abort_flag, g.dev_status)) return false;
         tc_fence_after();
         const uint32_t o_addr = tmem + 2 * BN + r * D, p_addr = tmem + r * BN + 64;
@@ -303,48 +335,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           umma_bf16_ts(o_addr, p_addr + kk * 8, dVs + (uint64_t)(kk * (2048 >> 4)), idesc_o,
-                       (js[r] > 1 || kk > 0) ? 1u : 0u);
-        umma_commit(pv_done + r);
-        pend[r] = false;
+                       (js > 1 || kk > 0) ? 1u : 0u);
+        if (js == (r ? kB : kA)) umma_commit(pv_done + r);  // the query tile's last P V
+        pend = false;
         return true;
+      };
+      // S = Q_r K^T for the K tile in ring slot st
+      auto issue_s = [&](auto rc, int st) {
+        constexpr int r = decltype(rc)::value;
+        const uint64_t dQr = dQ + (uint64_t)(r * (Lay::QB >> 4)), dKs = dK + (uint64_t)(st * (Lay::KB >> 4));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+          umma_bf16_ss(tmem + r * BN, dQr + off, dKs + off, idesc_s, kk > 0);
+        }
+        umma_commit(s_full + r);
+        (r ? js1 : js0)++;
+        (r ? pend1 : pend0) = true;
       };
       UnionWalk uw(listA, kA, listB, kB, nt, nullptr);
       int t, e = 0;
-      bool mem[2];
-      while (ok && uw.next(t, mem[0], mem[1])) {
+      bool mA, mB;
+      while (ok && uw.next(t, mA, mB)) {
         const int st = e % KST;
         if (!mbar_wait(k_full + st, (e / KST) & 1, abort_flag, g.dev_status)) break;
         tc_fence_after();
         // query tiles that kept tile e: finish their previous P V (P shares
         // the S columns), then S for tile e
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          if (!mem[r]) continue;
-          if (pend[r] && !(ok = issue_pv(r))) break;
-          const uint64_t dQr = dQ + (uint64_t)(r * (Lay::QB >> 4)), dKs = dK + (uint64_t)(st * (Lay::KB >> 4));
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
-            umma_bf16_ss(tmem + r * BN, dQr + off, dKs + off, idesc_s, kk > 0);
-          }
-          umma_commit(s_full + r);
-          js[r]++;
-          pend[r] = true;
+        if (mA) {
+          if (pend0 && !(ok = issue_pv(I0{}))) break;
+          issue_s(I0{}, st);
         }
-        if (!ok) break;
-        // the other query tile: release its P V of tile e-1 only now, so its
-        // softmax overlaps the S just issued
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-          if (!mem[r] && pend[r] && !(ok = issue_pv(r))) break;
-        if (!ok) break;
-        if (prev_e >= 0) umma_commit(v_empty + prev_e % VST);  // all P V of prev_e issued
-        umma_commit(k_empty + st);
+        if (mB) {
+          if (pend1 && !(ok = issue_pv(I1{}))) break;
+          issue_s(I1{}, st);
+        }
+        // a query tile that did not keep it: release its P V of tile e-1
+        // only now, so its softmax overlaps the S just issued
+        if (!mA && pend0 && !(ok = issue_pv(I0{}))) break;
+        if (!mB && pend1 && !(ok = issue_pv(I1{}))) break;
+        umma_commit(step_done + e % SDR);  // frees K of e and V of e-1 for the producers
         prev_e = e;
         ++e;
       }
-      for (int r = 0; r < 2 && ok; ++r)
-        if (pend[r]) ok = issue_pv(r);
+      if (ok && pend0) ok = issue_pv(I0{});
+      if (ok && pend1) ok = issue_pv(I1{});
       umma_commit(mma_drain);
       mbar_wait_drain(mma_drain, 0, VEDA_WAIT_LIMIT_NS);
     }
@@ -399,12 +434,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float m_new = redo ? fmaxf(m, mx2) : m;
         const float alpha = fast_exp2(m - m_new);
         if (j > 0) {
-          // O must hold P V of the previous tile before it is rescaled
-          if (!__all_sync(0xffffffffu, mbar_wait(pv_done + r, (j - 1) & 1, abort_flag, g.dev_status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+          // O already holds P V of the previous tile: the MMA thread issues
+          // it before this tile's S, and s_full tracks every MMA it issued
+          // before its commit
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -437,7 +469,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
         if (prm.lse) prm.lse[orow_i] = 0.f;
       }
-    } else if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done + r, (kr - 1) & 1, abort_flag, g.dev_status))) {
+    } else if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done + r, 0, abort_flag, g.dev_status))) {
       tc_fence_after();
       const float inv = row_valid ? 1.0f / l : 0.f;
       __nv_bfloat16* orow = prm.op + orow_i * D;
