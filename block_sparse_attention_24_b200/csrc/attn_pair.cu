@@ -59,13 +59,15 @@ struct PairLayout {
   static constexpr int OFF_BAR = OFF_V + VST * KB;
   // q_full, k_full[KST], v_full[VST], step_done[SDR], s_full[2], p_full[2], pv_done[2], drain
   static constexpr int NUM_BARS = 1 + KST + VST + SDR + 2 + 2 + 2 + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int SMEM_ALLOC = BYTES + 1024;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, list check
+  static constexpr int OFF_BM = (OFF_MISC + 16 + 15) / 16 * 16;  // kept-tile bitmaps of A and B
+  // dynamic shared memory for bitmaps of `words` 32-bit words each
+  static constexpr int alloc(int words) { return OFF_BM + 8 * words + 1024; }
 };
 
 struct PairParams {
   int32_t k_cap;
+  int32_t bm_words;  // 32-bit words per kept-tile bitmap in shared memory; 0: no bitmaps
   float scale_log2;
   const int32_t* idx;
   __nv_bfloat16* op;
@@ -124,6 +126,35 @@ struct UnionWalk {
       tb = ++ib < kb ? checked(rb, true) : INT_MAX;
       rb = raw(lb, ib + 1, kb);
     }
+    return true;
+  }
+};
+
+// The same walk over kept-tile bitmaps in shared memory (valid when both
+// lists are ascending, distinct and in range): the next union tile is the
+// lowest set bit of the two current words, so a step costs a few integer
+// instructions and no load except one shared word per 32 tiles.
+struct BitWalk {
+  const uint32_t* a;
+  const uint32_t* b;
+  int nw, wi;
+  uint32_t wa, wb;  // current words with the tiles already visited cleared
+  __device__ BitWalk(const uint32_t* a_, const uint32_t* b_, int nw_) : a(a_), b(b_), nw(nw_), wi(0), wa(0), wb(0) {
+    if (nw > 0) wa = a[0], wb = b[0];
+  }
+  __device__ bool next(int& t, bool& ma, bool& mb) {
+    while ((wa | wb) == 0u) {
+      if (++wi >= nw) return false;
+      wa = a[wi];
+      wb = b[wi];
+    }
+    const int pos = __ffs(wa | wb) - 1;
+    const uint32_t bit = 1u << pos;
+    ma = (wa & bit) != 0u;
+    mb = (wb & bit) != 0u;
+    wa &= ~bit;
+    wb &= ~bit;
+    t = wi * 32 + pos;
     return true;
   }
 };
@@ -241,6 +272,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* mma_drain = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
+  volatile int* list_bad = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 8);
+  uint32_t* bmA = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BM);
+  uint32_t* bmB = bmA + prm.bm_words;
+  const bool try_bm = prm.idx != nullptr && prm.bm_words > 0;  // uniform over the CTA
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < Lay::NUM_BARS; ++i) {
@@ -248,15 +283,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar, (bar == p_full || bar == p_full + 1) ? 128 : 1);
     }
     *abort_flag = 0;
+    *list_bad = 0;
     fence_mbar_init();
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
+  if (try_bm) {
+    // kept-tile bitmaps of both lists, built by all threads; an entry out of
+    // range or not above its predecessor leaves the CTA on the list merge
+    for (int i = threadIdx.x; i < 2 * prm.bm_words; i += NUM_THREADS) bmA[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < kA + kB; i += NUM_THREADS) {
+      const bool in_b = i >= kA;
+      const int32_t* l = in_b ? listB : listA;
+      const int j = in_b ? i - kA : i, kl = in_b ? kB : kA;
+      const int t = __ldg(l + j);
+      if (t < 0 || t >= nt || (j + 1 < kl && __ldg(l + j + 1) <= t)) *list_bad = 1;
+      else atomicOr((in_b ? bmB : bmA) + (t >> 5), 1u << (t & 31));
+    }
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const bool use_bm = try_bm && *list_bad == 0;
   if (warp >= 8) {
   regs_lower<REGS_ROLES>();
   if (warp == 8 || warp == 10) {
@@ -277,8 +328,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_3d(smem + Lay::OFF_Q + Lay::QB + bx * BM * 128, &tmQ, q_full, bx * 64, qbt * BM, bh);
         }
       }
-      UnionWalk uw(listA, kA, listB, kB, nt, is_k ? g.dev_status : nullptr);
-      int t, e = 0;
+      int e = 0;
+      // one instance per walk type, so only one walk's state is live
+      auto produce = [&](auto& uw) {
+      int t;
       bool ma, mb;
       while (uw.next(t, ma, mb)) {
         const int st = e % ST;
@@ -292,6 +345,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int bx = 0; bx < D / 64; ++bx)
           tma_load_3d(ring + st * Lay::KB + bx * BN * 128, map, full + st, bx * 64, t * BN, bh);
         ++e;
+      }
+      };
+      if (use_bm) {
+        BitWalk w(bmA, bmB, prm.bm_words);
+        produce(w);
+      } else {
+        UnionWalk w(listA, kA, listB, kB, nt, is_k ? g.dev_status : nullptr);
+        produce(w);
       }
       if (*abort_flag) {  // let every copy this warp started land before exiting
         if (is_k) mbar_wait_drain(q_full, 0, VEDA_WAIT_LIMIT_NS);
@@ -317,6 +378,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool pend0 = false, pend1 = false;  // a P V is pending
       int js0 = 0, js1 = 0;               // S issued
       int prev_e = -1;
+      int v_seen = -1;  // V ring entry already waited for
       bool ok = mbar_wait(q_full, 0, abort_flag, g.dev_status);
       if (ok) tc_fence_after();
       using I0 = std::integral_constant<int, 0>;
@@ -328,7 +390,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool& pend = r ? pend1 : pend0;
         const int vs = prev_e % VST;
         if (!mbar_wait(p_full + r, (js - 1) & 1, abort_flag, g.dev_status)) return false;
-        if (!mbar_wait(v_full + vs, (prev_e / VST) & 1, abort_flag, g.dev_status)) return false;
+        if (v_seen != prev_e) {  // both query tiles' P V of a shared tile read one V entry
+          if (!mbar_wait(v_full + vs, (prev_e / VST) & 1, abort_flag, g.dev_status)) return false;
+          v_seen = prev_e;
+        }
         tc_fence_after();
         const uint32_t o_addr = tmem + 2 * BN + r * D, p_addr = tmem + r * BN + 64;
         const uint64_t dVs = dV + (uint64_t)(vs * (Lay::KB >> 4));
@@ -353,7 +418,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         (r ? js1 : js0)++;
         (r ? pend1 : pend0) = true;
       };
-      UnionWalk uw(listA, kA, listB, kB, nt, nullptr);
+      // one instance per walk type, so only one walk's state is live
+      auto issue_all = [&](auto& uw) {
       int t, e = 0;
       bool mA, mB;
       while (ok && uw.next(t, mA, mB)) {
@@ -377,6 +443,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_commit(step_done + e % SDR);  // frees K of e and V of e-1 for the producers
         prev_e = e;
         ++e;
+      }
+      };
+      if (use_bm) {
+        BitWalk w(bmA, bmB, prm.bm_words);
+        issue_all(w);
+      } else {
+        UnionWalk w(listA, kA, listB, kB, nt, nullptr);
+        issue_all(w);
       }
       if (ok && pend0) ok = issue_pv(I0{});
       if (ok && pend1) ok = issue_pv(I1{});
@@ -507,11 +581,17 @@ cudaError_t launch_pair_t(const LayerGeom& g, const void* qp, const void* kp, co
   if (encode_tensor_map_3d_bf16(&tk, kp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (encode_tensor_map_3d_bf16(&tv, vp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   auto kern = sparse_attn_pair_kernel<D>;
-  const int smem = PairLayout<D>::SMEM_ALLOC;
+  PairParams p = prm;
+  p.bm_words = (g.nt_cap + 31) / 32;
+  int smem = PairLayout<D>::alloc(p.bm_words);
+  if (smem > 232448) {  // bitmaps do not fit beside the rings: list merge
+    p.bm_words = 0;
+    smem = PairLayout<D>::alloc(0);
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((g.nt_cap + 1) / 2, g.heads, g.B);
-  kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, tv, prm);
+  kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -523,6 +603,7 @@ cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const vo
                                     cudaStream_t s) {
   PairParams prm;
   prm.k_cap = k_cap;
+  prm.bm_words = 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.idx = idx;
   prm.op = reinterpret_cast<__nv_bfloat16*>(op);

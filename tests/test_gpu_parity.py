@@ -276,7 +276,7 @@ def test_topk_large_rows():
 
 # --------------------------------------------------------- sparse attention
 
-def _attention_case(w, k_override=None, dense=False, random_lists=True, key_tile_gain=None):
+def _attention_case(w, k_override=None, dense=False, random_lists=True, key_tile_gain=None, shuffle=False):
     L = _layer(w)
     lays, perms, n_cap, nt_cap = oracle_geometry(w)
     q, k, v = _inputs(w)
@@ -295,6 +295,10 @@ def _attention_case(w, k_override=None, dense=False, random_lists=True, key_tile
         for h in range(w.heads):
             nt = lays[h]["nt"]
             idx[b, h, :nt] = synth.random_index_lists(nt, nt, ks[h], k_cap, seed=100 * b + h + w.seed)
+            if shuffle:     # kept tiles in any order: the same attention
+                rng = np.random.default_rng(500 + 100 * b + h)
+                for a in range(nt):
+                    idx[b, h, a, :ks[h]] = rng.permutation(idx[b, h, a, :ks[h]])
     op = torch.empty_like(qp)
     lse = torch.empty((w.B, w.heads, n_cap), dtype=torch.float32, device=DEV)
     scale = 1 / math.sqrt(w.d)
@@ -321,6 +325,14 @@ def _attention_case(w, k_override=None, dense=False, random_lists=True, key_tile
 @pytest.mark.parametrize("name", list(WL))
 def test_sparse_attention_random_lists(name):
     _attention_case(WL[name])
+
+
+@pytest.mark.parametrize("name", ["ragged-d128-t128", "batch2-d64-t128", "odd-d128-t64"])
+def test_sparse_attention_unsorted_lists(name):
+    """Kept-tile lists in arbitrary order (the call does not require them
+    ascending): the kernel then merges the lists instead of walking its
+    kept-tile bitmaps, with the same result."""
+    _attention_case(WL[name], shuffle=True)
 
 
 @pytest.mark.parametrize("name", list(WL))
