@@ -159,6 +159,72 @@ struct BitWalk {
   }
 };
 
+// A third order over the same bitmaps, for heads whose tiles are all full
+// (then the softmax never needs to know which tile it holds, and each query
+// tile may take its kept tiles in any order). A union tile only one query
+// tile kept runs that query tile's chain alone: the next S can only follow
+// its own softmax and P V. So tiles only A kept and tiles only B kept are
+// taken alternately while both remain, letting each chain's latency hide
+// behind the other's work; otherwise the lowest remaining tile comes next.
+// Tiles both kept are steps of their own, as in the other walks.
+struct AltWalk {
+  struct Cursor {  // lowest remaining tile of one category (A only, B only, both)
+    int wi;
+    uint32_t w;
+  };
+  const uint32_t* a;
+  const uint32_t* b;
+  int nw;
+  Cursor ca, cb, cs;
+  int last;  // 1: the previous step was a tile only A kept, 2: only B, 0: otherwise
+  __device__ uint32_t word(int c, int wi) const {
+    const uint32_t x = a[wi], y = b[wi];
+    return c == 0 ? (x & ~y) : (c == 1 ? (y & ~x) : (x & y));
+  }
+  __device__ void init(Cursor& cu, int c) {
+    cu.wi = 0;
+    cu.w = nw > 0 ? word(c, 0) : 0u;
+  }
+  // tile index of the lowest remaining bit, INT_MAX when none is left
+  __device__ int head(Cursor& cu, int c) {
+    while (cu.w == 0u) {
+      if (cu.wi + 1 >= nw) return INT_MAX;
+      ++cu.wi;
+      cu.w = word(c, cu.wi);
+    }
+    return cu.wi * 32 + __ffs(cu.w) - 1;
+  }
+  __device__ AltWalk(const uint32_t* a_, const uint32_t* b_, int nw_) : a(a_), b(b_), nw(nw_), last(0) {
+    init(ca, 0);
+    init(cb, 1);
+    init(cs, 2);
+  }
+  __device__ bool next(int& t, bool& ma, bool& mb) {
+    const int ha = head(ca, 0), hb = head(cb, 1), hs = head(cs, 2);
+    int c;
+    if (last == 1 && hb != INT_MAX) c = 1;
+    else if (last == 2 && ha != INT_MAX) c = 0;
+    else if (ha == INT_MAX && hb == INT_MAX && hs == INT_MAX) return false;
+    else c = (ha < hb && ha < hs) ? 0 : (hb < hs ? 1 : 2);
+    // consume the lowest bit of the chosen category (explicit branches keep
+    // the cursors in registers)
+    if (c == 0) {
+      t = ha;
+      ca.w &= ca.w - 1u;
+    } else if (c == 1) {
+      t = hb;
+      cb.w &= cb.w - 1u;
+    } else {
+      t = hs;
+      cs.w &= cs.w - 1u;
+    }
+    ma = c != 1;
+    mb = c != 0;
+    last = c == 0 ? 1 : (c == 1 ? 2 : 0);
+    return true;
+  }
+};
+
 // Maximum of one 64-key half h of a row of S over the valid keys (all of
 // them unless !FULL, then keys below `klen`): eight 3-input max chains.
 template <bool FULL>
@@ -347,7 +413,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++e;
       }
       };
-      if (use_bm) {
+      if (use_bm && !hg.padded) {
+        AltWalk w(bmA, bmB, prm.bm_words);
+        produce(w);
+      } else if (use_bm) {
         BitWalk w(bmA, bmB, prm.bm_words);
         produce(w);
       } else {
@@ -445,7 +514,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++e;
       }
       };
-      if (use_bm) {
+      if (use_bm && !hg.padded) {
+        AltWalk w(bmA, bmB, prm.bm_words);
+        issue_all(w);
+      } else if (use_bm) {
         BitWalk w(bmA, bmB, prm.bm_words);
         issue_all(w);
       } else {

@@ -84,19 +84,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of the phase with parity `parity` (no suspension).
-__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // As mbar_try_wait, but lets the hardware suspend the thread for up to
 // `hint_ns` while the phase is incomplete; the thread resumes as soon as the
 // phase completes, so a long hint costs no latency and keeps a waiting warp
@@ -127,7 +114,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t pari
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int32_t* status, uint64_t limit_ns = VEDA_WAIT_LIMIT_NS) {
   const uint32_t addr = smem_u32(bar);
-  if (mbar_test_wait(addr, parity)) return true;
+  if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_sleep(addr, parity, VEDA_WAIT_HINT_NS)) return true;
