@@ -580,7 +580,7 @@ def main():
     ap.add_argument("--config", type=int, default=3)
     ap.add_argument("--keep", type=float, default=None)
     ap.add_argument("--dense-reps", type=int, default=2)
-    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=24)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
