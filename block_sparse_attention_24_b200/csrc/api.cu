@@ -247,14 +247,18 @@ int veda_tile_scores_topk(const veda_layer* L, const float* dq, const float* dk,
                       "veda_tile_scores_topk");
 }
 
-int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const void* vp, const int32_t* idx,
-                     const int32_t* k, int32_t k_cap, float scale, void* op, float* lse, cudaStream_t stream) {
+namespace {
+// Shared by veda_sparse_attn (permuted output `op`) and
+// veda_sparse_attn_unpermute (token-order output `o`).
+int sparse_attn_call(const veda_layer* L, const void* qp, const void* kp, const void* vp, const int32_t* idx,
+                     const int32_t* k, int32_t k_cap, float scale, void* out, bool to_tokens, float* lse,
+                     cudaStream_t stream, const char* name) {
   veda::LayerGeom g;
   VEDA_TRY(build_geom(L, &g));
   VEDA_TRY(check_ptr(qp, "qp"));
   VEDA_TRY(check_ptr(kp, "kp"));
   VEDA_TRY(check_ptr(vp, "vp"));
-  VEDA_TRY(check_ptr(op, "op"));
+  VEDA_TRY(check_ptr(out, to_tokens ? "o" : "op"));
   if (lse) VEDA_TRY(check_ptr(lse, "lse"));
   if (!(scale > 0.f) || scale != scale) return fail(VEDA_ERR_INVALID_ARG, "scale must be positive and finite");
   if (idx) {
@@ -271,8 +275,21 @@ int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const 
     for (int h = 0; h < g.heads; ++h) g.h[h].k = g.h[h].nt;
     k_cap = 0;
   }
-  return after_launch(veda::launch_sparse_attn(g, qp, kp, vp, idx, k_cap, scale, op, lse, stream),
-                      "veda_sparse_attn");
+  return after_launch(veda::launch_sparse_attn(g, qp, kp, vp, idx, k_cap, scale, to_tokens ? nullptr : out, lse,
+                                                stream, to_tokens ? out : nullptr),
+                      name);
+}
+}  // namespace
+
+int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const void* vp, const int32_t* idx,
+                     const int32_t* k, int32_t k_cap, float scale, void* op, float* lse, cudaStream_t stream) {
+  return sparse_attn_call(L, qp, kp, vp, idx, k, k_cap, scale, op, false, lse, stream, "veda_sparse_attn");
+}
+
+int veda_sparse_attn_unpermute(const veda_layer* L, const void* qp, const void* kp, const void* vp,
+                               const int32_t* idx, const int32_t* k, int32_t k_cap, float scale, void* o,
+                               float* lse, cudaStream_t stream) {
+  return sparse_attn_call(L, qp, kp, vp, idx, k, k_cap, scale, o, true, lse, stream, "veda_sparse_attn_unpermute");
 }
 
 size_t veda_full_attn_tilemax_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows) {

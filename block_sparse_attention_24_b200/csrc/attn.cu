@@ -58,7 +58,8 @@ struct AttnParams {
   int32_t k_cap;
   float scale_log2;  // scale * log2(e)
   const int32_t* idx;
-  __nv_bfloat16* op;
+  __nv_bfloat16* op;    // [B, heads, n_cap, D] (permuted order), or NULL when otok is set
+  __nv_bfloat16* otok;  // [B, N, heads, D] (token order) or NULL: rows written straight to their tokens
   float* lse;
 };
 
@@ -93,8 +94,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n_qb = (nt + NSUB - 1) / NSUB;
   const long long row0 = (long long)bh * g.n_cap + (long long)qb * BM;  // first output row
 
-  if (qb >= n_qb) {  // padding rows of this head: zero output
-    for (int i = threadIdx.x; i < BM * D / 8; i += NUM_THREADS) {
+  if (qb >= n_qb) {  // padding rows of this head: zero output (none in token order)
+    for (int i = threadIdx.x; prm.op && i < BM * D / 8; i += NUM_THREADS) {
       const int r = i / (D / 8);
       if (qb * BM + r < g.n_cap)
         reinterpret_cast<uint4*>(prm.op + (row0 + r) * D)[i % (D / 8)] = make_uint4(0, 0, 0, 0);
@@ -350,7 +351,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const float inv = row_valid ? 1.0f / l : 0.f;
       const bool in_range = qb * BM + r < g.n_cap;
-      __nv_bfloat16* orow = prm.op + (row0 + r) * D;
+      // the row's destination: its permuted slot, or its token (padding rows
+      // have none)
+      __nv_bfloat16* orow = nullptr;
+      if (prm.otok) {
+        const long long tok = row_valid ? tile_row_token(g, hg, a, r % TILE) : -1;
+        if (tok >= 0) orow = prm.otok + (((long long)b * g.T * g.H * g.W + tok) * g.heads + h) * D;
+      } else if (in_range) {
+        orow = prm.op + (row0 + r) * D;
+      }
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
@@ -359,7 +368,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           o[e] = pack_bf16x2_rn(__uint_as_float(u[2 * e]) * inv, __uint_as_float(u[2 * e + 1]) * inv);
-        if (in_range) {
+        if (orow) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
@@ -398,17 +407,19 @@ cudaError_t launch_t(const LayerGeom& g, const void* qp, const void* kp, const v
 
 cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                     const int32_t* idx, int k_cap, float scale, void* op, float* lse,
-                                    cudaStream_t s);
+                                    cudaStream_t s, void* o_tokens);
 
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
-                               const int32_t* idx, int k_cap, float scale, void* op, float* lse, cudaStream_t s) {
+                               const int32_t* idx, int k_cap, float scale, void* op, float* lse, cudaStream_t s,
+                               void* o_tokens) {
   AttnParams prm;
   prm.k_cap = k_cap;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.idx = idx;
-  prm.op = reinterpret_cast<__nv_bfloat16*>(op);
+  prm.op = o_tokens ? nullptr : reinterpret_cast<__nv_bfloat16*>(op);
+  prm.otok = reinterpret_cast<__nv_bfloat16*>(o_tokens);
   prm.lse = lse;
-  if (g.tile == 128) return launch_sparse_attn_pair(g, qp, kp, vp, idx, k_cap, scale, op, lse, s);
+  if (g.tile == 128) return launch_sparse_attn_pair(g, qp, kp, vp, idx, k_cap, scale, op, lse, s, o_tokens);
   if (g.d == 128) return launch_t<128, 64>(g, qp, kp, vp, prm, s);
   return launch_t<64, 64>(g, qp, kp, vp, prm, s);
 }

@@ -70,7 +70,8 @@ struct PairParams {
   int32_t bm_words;  // 32-bit words per kept-tile bitmap in shared memory; 0: no bitmaps
   float scale_log2;
   const int32_t* idx;
-  __nv_bfloat16* op;
+  __nv_bfloat16* op;    // [B, heads, n_cap, D] (permuted order), or NULL when otok is set
+  __nv_bfloat16* otok;  // [B, N, heads, D] (token order) or NULL: rows written straight to their tokens
   float* lse;
 };
 
@@ -310,8 +311,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int qa = 2 * cp, qbt = 2 * cp + 1;  // the two query tiles
   const long long rowA = (long long)bh * g.n_cap + (long long)qa * BM;
 
-  if (qa >= nt) {  // both query tiles are padding: zero output rows
-    for (int i = threadIdx.x; i < 2 * BM * D / 8; i += NUM_THREADS) {
+  if (qa >= nt) {  // both query tiles are padding: zero output rows (none in token order)
+    for (int i = threadIdx.x; prm.op && i < 2 * BM * D / 8; i += NUM_THREADS) {
       const int r = i / (D / 8);
       if (qa * BM + r < g.n_cap)
         reinterpret_cast<uint4*>(prm.op + (rowA + r) * D)[i % (D / 8)] = make_uint4(0, 0, 0, 0);
@@ -608,17 +609,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // epilogue: O / l -> bf16
     const long long orow_i = rowA + (long long)r * BM + row;
     const bool in_range = a * BM + row < g.n_cap;
-    if (kr == 0) {  // query tile beyond this head's tiles: zero rows
+    if (kr == 0) {  // query tile beyond this head's tiles: zero rows (none in token order)
       if (in_range) {
-        uint4* dst = reinterpret_cast<uint4*>(prm.op + orow_i * D);
+        if (prm.op) {
+          uint4* dst = reinterpret_cast<uint4*>(prm.op + orow_i * D);
 #pragma unroll
-        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+          for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+        }
         if (prm.lse) prm.lse[orow_i] = 0.f;
       }
     } else if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done + r, 0, abort_flag, g.dev_status))) {
       tc_fence_after();
       const float inv = row_valid ? 1.0f / l : 0.f;
-      __nv_bfloat16* orow = prm.op + orow_i * D;
+      // the row's destination: its permuted slot, or its token (padding rows
+      // have none)
+      __nv_bfloat16* orow = nullptr;
+      if (prm.otok) {
+        const long long n = row_valid ? tile_row_token(g, hg, a, row) : -1;
+        if (n >= 0) orow = prm.otok + (((long long)b * g.T * g.H * g.W + n) * g.heads + h) * D;
+      } else if (in_range) {
+        orow = prm.op + orow_i * D;
+      }
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
@@ -627,7 +638,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           o[e] = pack_bf16x2_rn(__uint_as_float(u[2 * e]) * inv, __uint_as_float(u[2 * e + 1]) * inv);
-        if (in_range) {
+        if (orow) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
@@ -672,13 +683,14 @@ cudaError_t launch_pair_t(const LayerGeom& g, const void* qp, const void* kp, co
 // 128-token tiles: two query tiles per CTA sharing the loads of their union.
 cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                     const int32_t* idx, int k_cap, float scale, void* op, float* lse,
-                                    cudaStream_t s) {
+                                    cudaStream_t s, void* o_tokens) {
   PairParams prm;
+  prm.otok = reinterpret_cast<__nv_bfloat16*>(o_tokens);
   prm.k_cap = k_cap;
   prm.bm_words = 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.idx = idx;
-  prm.op = reinterpret_cast<__nv_bfloat16*>(op);
+  prm.op = o_tokens ? nullptr : reinterpret_cast<__nv_bfloat16*>(op);
   prm.lse = lse;
   if (g.d == 128) return launch_pair_t<128>(g, qp, kp, vp, prm, s);
   return launch_pair_t<64>(g, qp, kp, vp, prm, s);

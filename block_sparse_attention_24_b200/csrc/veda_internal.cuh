@@ -43,6 +43,20 @@ __host__ __device__ inline int tile_len(const HeadGeom& g, int T, int t) {
   return steps * g.ph * g.pw;
 }
 
+// Token index n = (t*H + y)*W + x (within its batch element) of row `row`
+// of tile `a` of a head, or -1 for a padding row past T: the inverse of the
+// head-aware tiling permutation for one row.
+__host__ __device__ inline long long tile_row_token(const LayerGeom& g, const HeadGeom& hg, int a, int row) {
+  const int slab = hg.ph * hg.pw;
+  const int lt = row / slab, lr = row - lt * slab;
+  const int ly = lr / hg.pw, lx = lr - ly * hg.pw;
+  const int tt = a / hg.tps, rem = a - tt * hg.tps;
+  const int th = rem / hg.nwt, tw = rem - th * hg.nwt;
+  const int t = tt * hg.pt + lt;
+  if (t >= g.T) return -1;
+  return ((long long)t * g.H + th * hg.ph + ly) * g.W + tw * hg.pw + lx;
+}
+
 __device__ inline void report(int32_t* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
@@ -398,7 +412,7 @@ cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int3
                         cudaStream_t s);
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, int k_cap, float scale, void* op, float* lse,
-                               cudaStream_t s);
+                               cudaStream_t s, void* o_tokens = nullptr);
 cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int n_heads_sel, const int32_t* rows,
                               int n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,
                               cudaStream_t s);

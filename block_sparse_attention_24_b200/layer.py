@@ -18,7 +18,8 @@ from typing import Dict, List, Optional, Sequence
 import torch
 
 from . import (Layer, veda_estimator_grad, veda_estimator_grad_ws_bytes, veda_full_attn_tilemax,
-               veda_full_attn_tilemax_ws_bytes, veda_permute, veda_permute_trippool, veda_sparse_attn, veda_tile_scores,
+               veda_full_attn_tilemax_ws_bytes, veda_permute, veda_permute_trippool, veda_sparse_attn,
+               veda_sparse_attn_unpermute, veda_tile_scores,
                veda_tile_scores_ws_bytes, veda_topk_mask)
 
 
@@ -107,11 +108,17 @@ class VedaLayer:
         veda_topk_mask(L, self.scores, self.k, self.k_cap, self.idx, self.mask, stream=stream)
 
     def attend(self, stream=None, out: Optional[torch.Tensor] = None):
-        """Sparse attention and the inverse permutation into `out` (default:
-        the layer's own output buffer)."""
+        """Sparse attention with the output written in token order into `out`
+        (default: the layer's own output buffer): one kernel, the inverse
+        permutation fused into its epilogue."""
+        veda_sparse_attn_unpermute(self.L, self.qp, self.kp, self.vp, self.idx, self.k, self.k_cap, self.attn_scale,
+                                   self.o if out is None else out, stream=stream)
+
+    def attend_permuted(self, stream=None):
+        """Sparse attention into the permuted buffer `op` (one row per tile
+        slot, padding rows zero), as the separate inverse permutation reads it."""
         veda_sparse_attn(self.L, self.qp, self.kp, self.vp, self.idx, self.k, self.k_cap, self.attn_scale, self.op,
                          stream=stream)
-        veda_permute(self.L, self.o if out is None else out, self.op, inverse=True, stream=stream)
 
     def distill(self, stream=None):
         if self.maps is None:
@@ -143,7 +150,8 @@ class VedaLayer:
     def forward(self, q, k, v, stream=None, out: Optional[torch.Tensor] = None, marks=None):
         """One step of the hot path, in order on one stream. `marks` (optional
         dict of CUDA events) is recorded at the stage boundaries "start",
-        "front", "attn0", "attn1", "unpermute", "end". (Running the tile map
+        "front", "attn0", "attn1", "unpermute", "end" (the inverse permutation
+        is fused into attention, so "attn1" and "unpermute" coincide). (Running the tile map
         on a second stream beside the rest measured slower: the split map
         already fills every SM.)"""
         main = torch.cuda.current_stream(self.device) if stream is None else stream
@@ -156,10 +164,8 @@ class VedaLayer:
         self.front(q, k, v, main)
         mark("front")
         mark("attn0")
-        veda_sparse_attn(self.L, self.qp, self.kp, self.vp, self.idx, self.k, self.k_cap, self.attn_scale, self.op,
-                         stream=main)
+        self.attend(main, out)      # the inverse permutation is the attention epilogue's store
         mark("attn1")
-        veda_permute(self.L, self.o if out is None else out, self.op, inverse=True, stream=main)
         mark("unpermute")
         self.distill(main)
         mark("end")

@@ -176,6 +176,18 @@ int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const 
                      const int32_t* idx, const int32_t* k, int32_t k_cap, float scale,
                      void* op, float* lse, cudaStream_t stream);
 
+/* veda_sparse_attn followed by the inverse permutation (Veda summary 2.2: the
+ * output returns to token order), in one kernel: each output row is written
+ * straight to its token, so the permuted output is never stored and read
+ * back (the pages name tighter kernel fusion as future work). o: [B, N, heads,
+ * d] bf16, N = T*H*W, every row written; identical values to veda_sparse_attn
+ * followed by veda_permute(..., inverse=1). lse (may be NULL) keeps the
+ * permuted layout [B, heads, n_cap] of veda_sparse_attn. Other arguments and
+ * errors as in veda_sparse_attn. */
+int veda_sparse_attn_unpermute(const veda_layer* L, const void* qp, const void* kp, const void* vp,
+                               const int32_t* idx, const int32_t* k, int32_t k_cap, float scale,
+                               void* o, float* lse, cudaStream_t stream);
+
 /* Oracle tile map and distillation loss (Veda summary 2.1, Target
  * Construction and Optimization; 2.3, Training Efficiency): for the selected
  * heads heads_sel[0..n_heads_sel) (HOST array) and query tiles

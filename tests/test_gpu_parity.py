@@ -336,6 +336,43 @@ def test_sparse_attention_unsorted_lists(name):
 
 
 @pytest.mark.parametrize("name", list(WL))
+@pytest.mark.parametrize("dense", [False, True])
+def test_sparse_attention_unpermute_fused(name, dense):
+    """veda_sparse_attn_unpermute writes each output row straight to its
+    token: bit-identical to veda_sparse_attn followed by the inverse
+    permutation (every token written), the same lse."""
+    w = WL[name]
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, k, v = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    kp, _ = _permuted(L, w, k)
+    vp, _ = _permuted(L, w, v)
+    ks = oracle_k(w, lays)
+    k_cap = max(ks)
+    idx = np.full((w.B, w.heads, nt_cap, k_cap), -1, np.int32)
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt = lays[h]["nt"]
+            idx[b, h, :nt] = synth.random_index_lists(nt, nt, ks[h], k_cap, seed=300 + 100 * b + h + w.seed)
+    idx_d = None if dense else torch.from_numpy(idx).to(DEV)
+    args = (None, None, 0) if dense else (idx_d, ks, k_cap)
+    scale = 1 / math.sqrt(w.d)
+    op = torch.empty_like(qp)
+    lse1 = torch.empty((w.B, w.heads, n_cap), dtype=torch.float32, device=DEV)
+    V.veda_sparse_attn(L, qp, kp, vp, *args, scale, op, lse1)
+    o_sep = torch.full_like(q, 3.0)
+    V.veda_permute(L, o_sep, op, inverse=True)
+    o = torch.full_like(q, 7.0)                       # every token must be overwritten
+    lse2 = torch.empty_like(lse1)
+    V.veda_sparse_attn_unpermute(L, qp, kp, vp, *args, scale, o, lse2)
+    V.veda_check_status(L)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_sep)
+    assert torch.equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("name", list(WL))
 def test_sparse_attention_dense_path(name):
     _attention_case(WL[name], dense=True)
 
