@@ -27,7 +27,7 @@ VEDA_ERR_BAD_INDEX = -5
 
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
-            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_sparse_attn_unpermute", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes", "veda_tilemap_kl",
+            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_sparse_attn_unpermute", "veda_sparse_attn_tokens", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes", "veda_tilemap_kl",
             "veda_check_status",
             "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_output_sq_error", "veda_selftest_wait_timeout", "veda_last_error")
 
@@ -73,6 +73,7 @@ _lib.veda_topk_mask.argtypes = [_LP, _P, _P, _I, _P, _P, _P]
 _lib.veda_tile_scores_topk.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _P, _P, _P, _P]
 _lib.veda_sparse_attn.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
 _lib.veda_sparse_attn_unpermute.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
+_lib.veda_sparse_attn_tokens.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
 _lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P, _P, _P, _P, _P, _P]
 _lib.veda_full_attn_tilemax_ws_bytes.argtypes = [_LP, _I, _I]
 _lib.veda_tilemap_kl.argtypes = [_LP, _P, _I, _P, _I, _P, _P, _P, _P, _P]
@@ -218,6 +219,15 @@ def veda_sparse_attn_unpermute(layer: Layer, qp, kp, vp, idx: Optional[torch.Ten
     karr = _host_i32(k) if k is not None else None
     _check(_lib.veda_sparse_attn_unpermute(layer.ref, _ptr(qp), _ptr(kp), _ptr(vp), _ptr(idx), karr, int(k_cap),
                                            float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def veda_sparse_attn_tokens(layer: Layer, q, k, v, idx: Optional[torch.Tensor], kk: Optional[Sequence[int]],
+                            k_cap: int, scale: float, o: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                            stream=None):
+    """Sparse attention with q, k, v and o in token order [B, N, heads, d]."""
+    karr = _host_i32(kk) if kk is not None else None
+    _check(_lib.veda_sparse_attn_tokens(layer.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), karr, int(k_cap),
+                                        float(scale), _ptr(o), _ptr(lse), _stream(stream)))
 
 
 def veda_full_attn_tilemax(layer: Layer, qp, kp, heads_sel: Sequence[int], qtile_rows: Optional[torch.Tensor],

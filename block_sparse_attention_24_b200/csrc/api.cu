@@ -73,6 +73,7 @@ int build_geom(const veda_layer* L, veda::LayerGeom* g) {
     hg.nt = (int)nt;
     hg.k = 0;
     hg.padded = (L->T % t.pt) != 0;
+    hg.tmap = 0;
     if (nt > nt_cap) nt_cap = (int)nt;
     if (nt * L->tile > n_cap) n_cap = (int)(nt * L->tile);
   }
@@ -125,6 +126,50 @@ CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t 
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// One token-layout map (see TokenMaps) for tiling (pt, ph, pw).
+CUresult encode_tensor_map_tokens_bf16(CUtensorMap* map, const void* base, const LayerGeom& g, int pt, int ph,
+                                       int pw) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return CUDA_ERROR_NOT_FOUND;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  const cuuint64_t d = (cuuint64_t)g.d, hd = d * g.heads;
+  cuuint64_t dims[5] = {d, (cuuint64_t)g.heads, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T * g.B};
+  cuuint64_t strides[4] = {d * 2, hd * 2, hd * g.W * 2, hd * g.W * g.H * 2};  // bytes, dims 1..4
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)pw, (cuuint32_t)ph, (cuuint32_t)pt};
+  cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+cudaError_t build_token_maps(LayerGeom& g, const void* q, const void* k, const void* v, TokenMaps* maps) {
+  int n = 0, tp[VEDA_MAX_TILINGS][3];
+  for (int h = 0; h < g.heads; ++h) {
+    HeadGeom& hg = g.h[h];
+    int i = 0;
+    while (i < n && !(tp[i][0] == hg.pt && tp[i][1] == hg.ph && tp[i][2] == hg.pw)) ++i;
+    if (i == n) {
+      if (n == VEDA_MAX_TILINGS) return cudaErrorNotSupported;
+      tp[n][0] = hg.pt, tp[n][1] = hg.ph, tp[n][2] = hg.pw;
+      ++n;
+    }
+    hg.tmap = i;
+  }
+  for (int i = 0; i < n; ++i) {
+    if (encode_tensor_map_tokens_bf16(&maps->q[i], q, g, tp[i][0], tp[i][1], tp[i][2]) != CUDA_SUCCESS ||
+        encode_tensor_map_tokens_bf16(&maps->k[i], k, g, tp[i][0], tp[i][1], tp[i][2]) != CUDA_SUCCESS ||
+        (v && encode_tensor_map_tokens_bf16(&maps->v[i], v, g, tp[i][0], tp[i][1], tp[i][2]) != CUDA_SUCCESS))
+      return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace veda
@@ -252,7 +297,7 @@ namespace {
 // veda_sparse_attn_unpermute (token-order output `o`).
 int sparse_attn_call(const veda_layer* L, const void* qp, const void* kp, const void* vp, const int32_t* idx,
                      const int32_t* k, int32_t k_cap, float scale, void* out, bool to_tokens, float* lse,
-                     cudaStream_t stream, const char* name) {
+                     cudaStream_t stream, const char* name, bool tokens_in = false) {
   veda::LayerGeom g;
   VEDA_TRY(build_geom(L, &g));
   VEDA_TRY(check_ptr(qp, "qp"));
@@ -275,15 +320,23 @@ int sparse_attn_call(const veda_layer* L, const void* qp, const void* kp, const 
     for (int h = 0; h < g.heads; ++h) g.h[h].k = g.h[h].nt;
     k_cap = 0;
   }
-  return after_launch(veda::launch_sparse_attn(g, qp, kp, vp, idx, k_cap, scale, to_tokens ? nullptr : out, lse,
-                                                stream, to_tokens ? out : nullptr),
-                      name);
+  const cudaError_t e = veda::launch_sparse_attn(g, qp, kp, vp, idx, k_cap, scale, to_tokens ? nullptr : out, lse,
+                                                stream, to_tokens ? out : nullptr, tokens_in);
+  if (e == cudaErrorNotSupported)
+    return fail(VEDA_ERR_UNSUPPORTED, "%s: more than %d distinct tilings", name, VEDA_MAX_TILINGS);
+  return after_launch(e, name);
 }
 }  // namespace
 
 int veda_sparse_attn(const veda_layer* L, const void* qp, const void* kp, const void* vp, const int32_t* idx,
                      const int32_t* k, int32_t k_cap, float scale, void* op, float* lse, cudaStream_t stream) {
   return sparse_attn_call(L, qp, kp, vp, idx, k, k_cap, scale, op, false, lse, stream, "veda_sparse_attn");
+}
+
+int veda_sparse_attn_tokens(const veda_layer* L, const void* q, const void* k_in, const void* v, const int32_t* idx,
+                            const int32_t* k, int32_t k_cap, float scale, void* o, float* lse, cudaStream_t stream) {
+  return sparse_attn_call(L, q, k_in, v, idx, k, k_cap, scale, o, true, lse, stream, "veda_sparse_attn_tokens",
+                          true);
 }
 
 int veda_sparse_attn_unpermute(const veda_layer* L, const void* qp, const void* kp, const void* vp,

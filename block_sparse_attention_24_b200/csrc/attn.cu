@@ -27,6 +27,8 @@
 // Every mbarrier wait is bounded (VEDA_WAIT_LIMIT_NS); on expiry the CTA
 // records VEDA_ERR_TIMEOUT, drains the copies and MMAs it issued, frees its
 // TMEM and exits.
+#include <type_traits>
+
 #include "veda_internal.cuh"
 
 namespace veda {
@@ -75,10 +77,17 @@ __device__ __forceinline__ int key_tile(const int32_t* row, int j, int nt, int32
   return t;
 }
 
-template <int D, int TILE>
+// Tensor maps of the permuted layout [B*heads, n_cap, d] (Q boxes of 128
+// rows, K/V boxes of one tile).
+struct PermMaps {
+  CUtensorMap q, k, v;
+};
+
+// TOK: Q, K, V in token order through the per-tiling 5D maps (TokenMaps).
+template <int D, int TILE, bool TOK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    sparse_attn_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ CUtensorMap tmQ,
-                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    sparse_attn_kernel(const __grid_constant__ LayerGeom g,
+                       const __grid_constant__ std::conditional_t<TOK, TokenMaps, PermMaps> maps,
                        const AttnParams prm) {
   using Lay = AttnLayout<D>;
   constexpr int NSUB = BM / TILE;
@@ -149,17 +158,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ----------------------------------------------------------- producers
     if (lane == 0) {
       const bool is_k = warp == 4;
-      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      const CUtensorMap* map;
+      const CUtensorMap* qmap;
+      if constexpr (TOK) {
+        map = is_k ? &maps.k[hg.tmap] : &maps.v[hg.tmap];
+        qmap = &maps.q[hg.tmap];
+      } else {
+        map = is_k ? &maps.k : &maps.v;
+        qmap = &maps.q;
+      }
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       uint8_t* ring = smem + (is_k ? Lay::OFF_K : Lay::OFF_V);
       constexpr int ST = KST;  // == VST
       tma_prefetch_desc(map);
       if (is_k) {
-        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(qmap);
         mbar_expect_tx(q_full, Lay::QB);
 #pragma unroll
-        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(sQ + bx * BM * 128, &tmQ, q_full, bx * 64, qb * BM, bh);
+        for (int bx = 0; bx < D / 64; ++bx) {
+          if constexpr (TOK) {
+#pragma unroll
+            for (int u = 0; u < NSUB; ++u)  // the block's query tiles, one box each
+              tma_load_tile_tokens(sQ + bx * BM * 128 + u * TILE * 128, qmap, q_full, g, hg, bx * 64, h, b,
+                                   qb * NSUB + u);
+          } else {
+            tma_load_3d(sQ + bx * BM * 128, qmap, q_full, bx * 64, qb * BM, bh);
+          }
+        }
       }
       int issued = 0;
       for (int t = 0; t < n; ++t) {
@@ -174,7 +200,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int u = 0; u < NSUB; ++u)
 #pragma unroll
           for (int bx = 0; bx < D / 64; ++bx)
-            tma_load_3d(dst + bx * BN * 128 + u * TILE * 128, map, full + st, bx * 64, kts[u] * TILE, bh);
+            if constexpr (TOK)
+              tma_load_tile_tokens(dst + bx * BN * 128 + u * TILE * 128, map, full + st, g, hg, bx * 64, h, b,
+                                   kts[u]);
+            else
+              tma_load_3d(dst + bx * BN * 128 + u * TILE * 128, map, full + st, bx * 64, kts[u] * TILE, bh);
         issued = t + 1;
       }
       if (*abort_flag) {  // let every copy this warp started land before exiting
@@ -385,21 +415,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int D, int TILE>
-cudaError_t launch_t(const LayerGeom& g, const void* qp, const void* kp, const void* vp, const AttnParams& prm,
+template <int D, int TILE, bool TOK>
+cudaError_t launch_t(const LayerGeom& g0, const void* qp, const void* kp, const void* vp, const AttnParams& prm,
                      cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
-  const uint64_t rows = (uint64_t)g.n_cap, planes = (uint64_t)g.B * g.heads;
-  if (encode_tensor_map_3d_bf16(&tq, qp, D, rows, planes, 64, BM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tensor_map_3d_bf16(&tk, kp, D, rows, planes, 64, TILE) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tensor_map_3d_bf16(&tv, vp, D, rows, planes, 64, TILE) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = sparse_attn_kernel<D, TILE>;
+  LayerGeom g = g0;
+  std::conditional_t<TOK, TokenMaps, PermMaps> maps;
+  if constexpr (TOK) {
+    const cudaError_t e = build_token_maps(g, qp, kp, vp, &maps);
+    if (e != cudaSuccess) return e;
+  } else {
+    const uint64_t rows = (uint64_t)g.n_cap, planes = (uint64_t)g.B * g.heads;
+    if (encode_tensor_map_3d_bf16(&maps.q, qp, D, rows, planes, 64, BM) != CUDA_SUCCESS ||
+        encode_tensor_map_3d_bf16(&maps.k, kp, D, rows, planes, 64, TILE) != CUDA_SUCCESS ||
+        encode_tensor_map_3d_bf16(&maps.v, vp, D, rows, planes, 64, TILE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  auto kern = sparse_attn_kernel<D, TILE, TOK>;
   const int smem = AttnLayout<D>::SMEM_ALLOC;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int qblocks = (g.nt_cap * TILE + BM - 1) / BM;
   const dim3 grid(qblocks, g.heads, g.B);
-  kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, tv, prm);
+  kern<<<grid, NUM_THREADS, smem, s>>>(g, maps, prm);
   return cudaGetLastError();
 }
 
@@ -407,11 +444,11 @@ cudaError_t launch_t(const LayerGeom& g, const void* qp, const void* kp, const v
 
 cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                     const int32_t* idx, int k_cap, float scale, void* op, float* lse,
-                                    cudaStream_t s, void* o_tokens);
+                                    cudaStream_t s, void* o_tokens, bool tokens_in);
 
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, int k_cap, float scale, void* op, float* lse, cudaStream_t s,
-                               void* o_tokens) {
+                               void* o_tokens, bool tokens_in) {
   AttnParams prm;
   prm.k_cap = k_cap;
   prm.scale_log2 = scale * 1.4426950408889634f;
@@ -419,9 +456,14 @@ cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* k
   prm.op = o_tokens ? nullptr : reinterpret_cast<__nv_bfloat16*>(op);
   prm.otok = reinterpret_cast<__nv_bfloat16*>(o_tokens);
   prm.lse = lse;
-  if (g.tile == 128) return launch_sparse_attn_pair(g, qp, kp, vp, idx, k_cap, scale, op, lse, s, o_tokens);
-  if (g.d == 128) return launch_t<128, 64>(g, qp, kp, vp, prm, s);
-  return launch_t<64, 64>(g, qp, kp, vp, prm, s);
+  if (g.tile == 128) return launch_sparse_attn_pair(g, qp, kp, vp, idx, k_cap, scale, op, lse, s, o_tokens, tokens_in);
+  if (tokens_in) {
+    if (!o_tokens) return cudaErrorInvalidValue;
+    if (g.d == 128) return launch_t<128, 64, true>(g, qp, kp, vp, prm, s);
+    return launch_t<64, 64, true>(g, qp, kp, vp, prm, s);
+  }
+  if (g.d == 128) return launch_t<128, 64, false>(g, qp, kp, vp, prm, s);
+  return launch_t<64, 64, false>(g, qp, kp, vp, prm, s);
 }
 
 }  // namespace veda

@@ -293,10 +293,17 @@ __device__ __forceinline__ float row_p(const uint32_t (&u)[BN], int klen, uint64
   return lo + hi;
 }
 
-template <int D>
+// Tensor maps of the permuted layout [B*heads, n_cap, d]: a tile is rows
+// [a*128, a*128+128) of plane b*heads + h.
+struct PermMaps {
+  CUtensorMap q, k, v;
+};
+
+// TOK: Q, K, V in token order through the per-tiling 5D maps (TokenMaps).
+template <int D, bool TOK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    sparse_attn_pair_kernel(const __grid_constant__ LayerGeom g, const __grid_constant__ CUtensorMap tmQ,
-                            const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    sparse_attn_pair_kernel(const __grid_constant__ LayerGeom g,
+                            const __grid_constant__ std::conditional_t<TOK, TokenMaps, PermMaps> maps,
                             const PairParams prm) {
   using Lay = PairLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -381,18 +388,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ----------------------------------------------------------- producers
     if (lane == 0) {
       const bool is_k = warp == 8;
-      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      const CUtensorMap* map;
+      const CUtensorMap* qmap;
+      if constexpr (TOK) {
+        map = is_k ? &maps.k[hg.tmap] : &maps.v[hg.tmap];
+        qmap = &maps.q[hg.tmap];
+      } else {
+        map = is_k ? &maps.k : &maps.v;
+        qmap = &maps.q;
+      }
+      // columns [bx*64, bx*64+64) of the 128 rows of tile a
+      auto load_tile = [&](void* dst, const CUtensorMap* m, uint64_t* bar, int bx, int a) {
+        if constexpr (TOK) tma_load_tile_tokens(dst, m, bar, g, hg, bx * 64, h, b, a);
+        else tma_load_3d(dst, m, bar, bx * 64, a * BN, bh);
+      };
       uint64_t* full = is_k ? k_full : v_full;
       const int ST = is_k ? KST : VST;
       uint8_t* ring = smem + (is_k ? Lay::OFF_K : Lay::OFF_V);
       tma_prefetch_desc(map);
       if (is_k) {
-        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(qmap);
         mbar_expect_tx(q_full, 2 * Lay::QB);
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_3d(smem + Lay::OFF_Q + bx * BM * 128, &tmQ, q_full, bx * 64, qa * BM, bh);
-          tma_load_3d(smem + Lay::OFF_Q + Lay::QB + bx * BM * 128, &tmQ, q_full, bx * 64, qbt * BM, bh);
+          load_tile(smem + Lay::OFF_Q + bx * BM * 128, qmap, q_full, bx, qa);
+          load_tile(smem + Lay::OFF_Q + Lay::QB + bx * BM * 128, qmap, q_full, bx, qbt);
         }
       }
       int e = 0;
@@ -410,7 +430,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_expect_tx(full + st, Lay::KB);
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_3d(ring + st * Lay::KB + bx * BN * 128, map, full + st, bx * 64, t * BN, bh);
+          load_tile(ring + st * Lay::KB + bx * BN * 128, map, full + st, bx, t);
         ++e;
       }
       };
@@ -655,15 +675,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int D>
-cudaError_t launch_pair_t(const LayerGeom& g, const void* qp, const void* kp, const void* vp, const PairParams& prm,
+template <int D, bool TOK>
+cudaError_t launch_pair_t(const LayerGeom& g0, const void* qp, const void* kp, const void* vp, const PairParams& prm,
                           cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
-  const uint64_t rows = (uint64_t)g.n_cap, planes = (uint64_t)g.B * g.heads;
-  if (encode_tensor_map_3d_bf16(&tq, qp, D, rows, planes, 64, BM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tensor_map_3d_bf16(&tk, kp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tensor_map_3d_bf16(&tv, vp, D, rows, planes, 64, BN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = sparse_attn_pair_kernel<D>;
+  LayerGeom g = g0;
+  std::conditional_t<TOK, TokenMaps, PermMaps> maps;
+  if constexpr (TOK) {
+    const cudaError_t e = build_token_maps(g, qp, kp, vp, &maps);
+    if (e != cudaSuccess) return e;
+  } else {
+    const uint64_t rows = (uint64_t)g.n_cap, planes = (uint64_t)g.B * g.heads;
+    if (encode_tensor_map_3d_bf16(&maps.q, qp, D, rows, planes, 64, BM) != CUDA_SUCCESS ||
+        encode_tensor_map_3d_bf16(&maps.k, kp, D, rows, planes, 64, BN) != CUDA_SUCCESS ||
+        encode_tensor_map_3d_bf16(&maps.v, vp, D, rows, planes, 64, BN) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  auto kern = sparse_attn_pair_kernel<D, TOK>;
   PairParams p = prm;
   p.bm_words = (g.nt_cap + 31) / 32;
   int smem = PairLayout<D>::alloc(p.bm_words);
@@ -674,16 +701,18 @@ cudaError_t launch_pair_t(const LayerGeom& g, const void* qp, const void* kp, co
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((g.nt_cap + 1) / 2, g.heads, g.B);
-  kern<<<grid, NUM_THREADS, smem, s>>>(g, tq, tk, tv, p);
+  kern<<<grid, NUM_THREADS, smem, s>>>(g, maps, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 // 128-token tiles: two query tiles per CTA sharing the loads of their union.
+// tokens_in: qp, kp, vp are in token order [B, N, heads, d] (then o_tokens is
+// the output).
 cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                     const int32_t* idx, int k_cap, float scale, void* op, float* lse,
-                                    cudaStream_t s, void* o_tokens) {
+                                    cudaStream_t s, void* o_tokens, bool tokens_in) {
   PairParams prm;
   prm.otok = reinterpret_cast<__nv_bfloat16*>(o_tokens);
   prm.k_cap = k_cap;
@@ -692,8 +721,13 @@ cudaError_t launch_sparse_attn_pair(const LayerGeom& g, const void* qp, const vo
   prm.idx = idx;
   prm.op = o_tokens ? nullptr : reinterpret_cast<__nv_bfloat16*>(op);
   prm.lse = lse;
-  if (g.d == 128) return launch_pair_t<128>(g, qp, kp, vp, prm, s);
-  return launch_pair_t<64>(g, qp, kp, vp, prm, s);
+  if (tokens_in) {
+    if (!o_tokens) return cudaErrorInvalidValue;
+    if (g.d == 128) return launch_pair_t<128, true>(g, qp, kp, vp, prm, s);
+    return launch_pair_t<64, true>(g, qp, kp, vp, prm, s);
+  }
+  if (g.d == 128) return launch_pair_t<128, false>(g, qp, kp, vp, prm, s);
+  return launch_pair_t<64, false>(g, qp, kp, vp, prm, s);
 }
 
 }  // namespace veda

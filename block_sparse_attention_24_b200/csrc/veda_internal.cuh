@@ -13,6 +13,7 @@
 
 #define VEDA_MAX_HEADS 128
 #define VEDA_MAX_NT 8192
+#define VEDA_MAX_TILINGS 8  // distinct tilings per layer on the token-layout path
 
 namespace veda {
 
@@ -25,6 +26,7 @@ struct HeadGeom {
   int32_t nwt;     // tiles along W = W/pw
   int32_t k;       // kept key tiles per query tile (attention / top-k)
   int32_t padded;  // 1 if p_t does not divide T (the last time slab of tiles is partial)
+  int32_t tmap;    // token-layout path: index of this head's tiling among the layer's tensor maps
 };
 
 struct LayerGeom {
@@ -168,6 +170,37 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_5d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+
+// Token-layout tensor maps. A tensor [B, N, heads, d] with N = T*H*W viewed
+// as 5D (d, heads, W, H, B*T); one map per distinct tiling (p_t, p_h, p_w)
+// whose box (64, 1, p_w, p_h, p_t) is one tile's rows, 64 columns, in the
+// tiling's in-tile order (row-major over t, y, x): a tile of the permuted
+// layout, gathered by TMA from token order. Rows past T read as zeros at the
+// tensor's end (and as the next batch element's rows inside it, which every
+// consumer masks as padding).
+struct TokenMaps {
+  CUtensorMap q[VEDA_MAX_TILINGS];
+  CUtensorMap k[VEDA_MAX_TILINGS];
+  CUtensorMap v[VEDA_MAX_TILINGS];
+};
+
+// Rows of tile `a` of head h, batch b, columns [c0, c0 + 64), from a token map.
+__device__ __forceinline__ void tma_load_tile_tokens(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                                     const LayerGeom& g, const HeadGeom& hg, int c0, int h, int b,
+                                                     int a) {
+  const int tt = a / hg.tps, rem = a - tt * hg.tps;
+  const int th = rem / hg.nwt, tw = rem - th * hg.nwt;
+  tma_load_5d(smem_dst, map, bar, c0, h, tw * hg.pw, th * hg.ph, b * g.T + tt * hg.pt);
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -412,7 +445,10 @@ cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int3
                         cudaStream_t s);
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, int k_cap, float scale, void* op, float* lse,
-                               cudaStream_t s, void* o_tokens = nullptr);
+                               cudaStream_t s, void* o_tokens = nullptr, bool tokens_in = false);
+// Token maps for Q, K (and V when non-NULL) of every distinct tiling; sets
+// each head's tmap. cudaErrorNotSupported past VEDA_MAX_TILINGS tilings.
+cudaError_t build_token_maps(LayerGeom& g, const void* q, const void* k, const void* v, TokenMaps* maps);
 cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int n_heads_sel, const int32_t* rows,
                               int n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,
                               cudaStream_t s);

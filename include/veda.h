@@ -188,6 +188,19 @@ int veda_sparse_attn_unpermute(const veda_layer* L, const void* qp, const void* 
                                const int32_t* idx, const int32_t* k, int32_t k_cap, float scale,
                                void* o, float* lse, cudaStream_t stream);
 
+/* Tile-skipping sparse attention with no permuted copies at all (Veda summary
+ * 2.2 and 2.3): q, k, v and o are in token order [B, N, heads, d] bf16. Each
+ * tile of the head-aware tiling is gathered by TMA straight from token order
+ * (one 5D tensor map per distinct tiling, whose box is the tile's rows in the
+ * tiling's in-tile order), and each output row is written to its token. The
+ * values equal those of veda_permute on q, k, v, veda_sparse_attn and the
+ * inverse veda_permute. idx, k, k_cap, scale as in veda_sparse_attn; lse (may
+ * be NULL) has the permuted layout [B, heads, n_cap]. At most 8 distinct
+ * tilings per layer (VEDA_ERR_UNSUPPORTED beyond). */
+int veda_sparse_attn_tokens(const veda_layer* L, const void* q, const void* k_in, const void* v,
+                            const int32_t* idx, const int32_t* k, int32_t k_cap, float scale,
+                            void* o, float* lse, cudaStream_t stream);
+
 /* Oracle tile map and distillation loss (Veda summary 2.1, Target
  * Construction and Optimization; 2.3, Training Efficiency): for the selected
  * heads heads_sel[0..n_heads_sel) (HOST array) and query tiles

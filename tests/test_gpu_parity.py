@@ -340,7 +340,8 @@ def test_sparse_attention_unsorted_lists(name):
 def test_sparse_attention_unpermute_fused(name, dense):
     """veda_sparse_attn_unpermute writes each output row straight to its
     token: bit-identical to veda_sparse_attn followed by the inverse
-    permutation (every token written), the same lse."""
+    permutation (every token written), the same lse. veda_sparse_attn_tokens
+    (Q, K, V gathered from token order by TMA) gives the same output and lse."""
     w = WL[name]
     L = _layer(w)
     lays, perms, n_cap, nt_cap = oracle_geometry(w)
@@ -366,10 +367,16 @@ def test_sparse_attention_unpermute_fused(name, dense):
     o = torch.full_like(q, 7.0)                       # every token must be overwritten
     lse2 = torch.empty_like(lse1)
     V.veda_sparse_attn_unpermute(L, qp, kp, vp, *args, scale, o, lse2)
+    # and with no permuted copies at all: tiles gathered by TMA from token order
+    o3 = torch.full_like(q, 5.0)
+    lse3 = torch.empty_like(lse1)
+    V.veda_sparse_attn_tokens(L, q, k, v, *args, scale, o3, lse3)
     V.veda_check_status(L)
     torch.cuda.synchronize()
     assert torch.equal(o, o_sep)
     assert torch.equal(lse1, lse2)
+    assert torch.equal(o3, o_sep)
+    assert torch.equal(lse3, lse1)          # padding rows are 0 on both paths
 
 
 @pytest.mark.parametrize("name", list(WL))
