@@ -3,13 +3,16 @@
 // key/value tiles are loaded; here each loaded tile also serves both query
 // tiles of the CTA when both kept it).
 //
-// A CTA owns query tiles A = 2c and B = 2c+1 of one head. Their kept-tile
-// lists are merged into one ascending sequence (the union); every union tile
-// is loaded by TMA exactly once, and S = Q K^T / O += P V are issued only for
-// the query tile(s) that kept it. Neighbouring query tiles keep mostly the
-// same key tiles (spatio-temporal locality), so the union is much shorter
-// than the two lists together and each K/V byte from L2 feeds up to twice the
-// tensor work of a one-tile CTA.
+// A CTA owns query tiles A = 2c and B = 2c+1 of one head. Every tile of the
+// union of their kept lists is loaded by TMA exactly once, and S = Q K^T /
+// O += P V are issued only for the query tile(s) that kept it. Neighbouring
+// query tiles keep mostly the same key tiles (spatio-temporal locality), so
+// the union is much shorter than the two lists together and each K/V byte
+// from L2 feeds up to twice the tensor work of a one-tile CTA. The union is
+// walked over kept-tile bitmaps built in shared memory (AltWalk), taking the
+// tiles only A kept and the tiles only B kept alternately where a head has
+// no padded tiles; lists that are not ascending and distinct are merged as
+// given (UnionWalk).
 //
 // Roles (384 threads):
 //   warps 0-3 / 4-7  softmax of query tile A / B: thread owns one row (TMEM
@@ -22,10 +25,15 @@
 //   warp 11          idle
 // MMA order per union tile e: for each query tile that kept e: its P V of
 // the previous union tile (if it kept that one), then S for e; then for a
-// query tile that did not keep e, its pending P V.
-// So one query tile's softmax runs while the tensor core works for the
-// other, and the V slot of every union tile is released one step later, in
-// order (no ring can fill with tiles whose consumer is far ahead).
+// query tile that did not keep e, its pending P V. So one query tile's
+// softmax runs while the tensor core works for the other. One commit per
+// union tile to a ring of step barriers frees the K slot of that tile and the
+// V slot of the one before.
+//
+// Q, K, V come either from the permuted layout [B, heads, n_cap, d] (3D
+// tensor maps) or straight from token order [B, N, heads, d] (TOK: 5D maps,
+// one per distinct tiling, whose box is a tile). The output goes to the
+// permuted layout or to each row's token.
 //
 // Every mbarrier wait is bounded (VEDA_WAIT_LIMIT_NS); on expiry the CTA
 // records VEDA_ERR_TIMEOUT, drains what it issued, frees its TMEM and exits.
@@ -74,18 +82,6 @@ struct PairParams {
   __nv_bfloat16* otok;  // [B, N, heads, D] (token order) or NULL: rows written straight to their tokens
   float* lse;
 };
-
-// j-th kept tile of a list (dense path: j), clamped into [0, nt); an
-// out-of-range entry is reported when `status` is given.
-__device__ __forceinline__ int list_tile(const int32_t* row, int j, int nt, int32_t* status) {
-  if (!row) return j;
-  int t = __ldg(row + j);
-  if (t < 0 || t >= nt) {
-    if (status) report(status, VEDA_ERR_BAD_INDEX);
-    t = 0;
-  }
-  return t;
-}
 
 // Walks the merge of two kept-tile lists: each call yields the next tile and
 // which of the two query tiles kept it. Every entry of both lists is visited
