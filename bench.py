@@ -459,6 +459,7 @@ def cpu_baseline(w, layer, L, budget_s):
     h = 0
     lens = O.head_layout(w.T, w.H, w.W, w.tilings[h])["lens"]
     f = lambda t: t[0, h].float().cpu().double().numpy()
+    torch.cuda.synchronize()    # the layer permutes V on its side stream
     qp, kp, vp = f(layer.qp), f(layer.kp), f(layer.vp)
     idx = layer.idx[0, h].cpu().numpy()
     flops, secs, tiles = oracle_attention_sample(w, qp, kp, vp, idx, layer.k[h], lens, budget_s)
