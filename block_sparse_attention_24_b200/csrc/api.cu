@@ -300,9 +300,9 @@ int sparse_attn_call(const veda_layer* L, const void* qp, const void* kp, const 
                      cudaStream_t stream, const char* name, bool tokens_in = false) {
   veda::LayerGeom g;
   VEDA_TRY(build_geom(L, &g));
-  VEDA_TRY(check_ptr(qp, "qp"));
-  VEDA_TRY(check_ptr(kp, "kp"));
-  VEDA_TRY(check_ptr(vp, "vp"));
+  VEDA_TRY(check_ptr(qp, tokens_in ? "q" : "qp"));
+  VEDA_TRY(check_ptr(kp, tokens_in ? "k" : "kp"));
+  VEDA_TRY(check_ptr(vp, tokens_in ? "v" : "vp"));
   VEDA_TRY(check_ptr(out, to_tokens ? "o" : "op"));
   if (lse) VEDA_TRY(check_ptr(lse, "lse"));
   if (!(scale > 0.f) || scale != scale) return fail(VEDA_ERR_INVALID_ARG, "scale must be positive and finite");
