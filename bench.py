@@ -226,6 +226,7 @@ def run_ours(args, world, rank, local):
     # per-stage breakdown of the front end (separate, untimed-for-value pass)
     stage_ms = stage_breakdown(V, L, layer, q, k, v, stream)
     grad_ms = estimator_grad_ms(layer, stream)
+    cache_ms = score_cache_ms(layer, q, k, v, stream)
 
     # dense path (same kernel, every tile kept) on the same permuted tensors
     dense_out = torch.empty_like(layer.op)
@@ -264,6 +265,7 @@ def run_ours(args, world, rank, local):
         "stage_ms": {**stage_ms, "front_end": round(front_ms, 3), "sparse_attn": round(attn_ms, 3),
                      "unpermute": round(unperm_ms, 3), "tilemap_kl": round(tail_ms, 3)},
         "estimator_grad_ms": grad_ms,
+        "score_cache": cache_ms,
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": sustained, "unit": UNIT,
                      "frac": round(attn_tflops / sustained, 4), "traffic": traffic,
                      "kernel": "sparse_attn_pair_kernel<128>",
@@ -299,6 +301,38 @@ def stage_breakdown(V, L, layer, q, k, v, stream):
     ev[4].record(stream)
     torch.cuda.synchronize()
     return {n: round(ev[i].elapsed_time(ev[i + 1]), 3) for i, n in enumerate(names)}
+
+
+def score_cache_ms(layer, q, k, v, stream, reps=5):
+    """Front end (Q/K permute + TripPool, V permute, then the scores and
+    top-k) with temporal caching of tile scores: every head rebuilt (ages
+    reset) vs every head reused (the same inputs again), plus the cache step
+    alone. The benchmark's own step does not cache."""
+    layer.enable_score_cache(0.05, 1 << 30)
+    layer.front(q, k, v)
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ms = []
+        for _ in range(reps):
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return round(statistics.median(ms), 3)
+
+    def rebuilt():
+        layer.cache_age.fill_(-1)
+        layer.front(q, k, v)
+
+    out = {"front_ms_rebuilt": timed(rebuilt), "front_ms_reused": timed(lambda: layer.front(q, k, v))}
+    import block_sparse_attention_24_b200 as V
+    out["cache_step_ms"] = timed(lambda: V.veda_score_cache_step(layer.L, layer.dq, layer.dk, layer.dq_ref, layer.dk_ref,
+                                                                 0.05, 1 << 30, layer.cache_age, layer.refresh,
+                                                                 layer.cache_ws))
+    layer.score_cache = None
+    return out
 
 
 def estimator_grad_ms(layer, stream, reps=5):

@@ -27,7 +27,7 @@ VEDA_ERR_BAD_INDEX = -5
 
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
-            "veda_topk_mask", "veda_tile_scores_topk", "veda_sparse_attn", "veda_sparse_attn_unpermute", "veda_sparse_attn_tokens", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes", "veda_tilemap_kl",
+            "veda_topk_mask", "veda_tile_scores_topk", "veda_tile_scores_heads", "veda_topk_mask_heads", "veda_score_cache_step", "veda_score_cache_ws_bytes", "veda_sparse_attn", "veda_sparse_attn_unpermute", "veda_sparse_attn_tokens", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes", "veda_tilemap_kl",
             "veda_check_status",
             "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_output_sq_error", "veda_selftest_wait_timeout", "veda_last_error")
 
@@ -70,6 +70,11 @@ _lib.veda_tile_scores_noalloc.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _P
 _lib.veda_tile_scores_ws_bytes.argtypes = [_LP, _I]
 _lib.veda_tile_scores_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_topk_mask.argtypes = [_LP, _P, _P, _I, _P, _P, _P]
+_lib.veda_tile_scores_heads.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _P, _P, _P]
+_lib.veda_topk_mask_heads.argtypes = [_LP, _P, _P, _I, _P, _P, _P, _P]
+_lib.veda_score_cache_step.argtypes = [_LP, _P, _P, _P, _P, _F, _I, _P, _P, _P, _P]
+_lib.veda_score_cache_ws_bytes.argtypes = [_LP]
+_lib.veda_score_cache_ws_bytes.restype = ctypes.c_size_t
 _lib.veda_tile_scores_topk.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _P, _P, _P, _P]
 _lib.veda_sparse_attn.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
 _lib.veda_sparse_attn_unpermute.argtypes = [_LP, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P]
@@ -195,6 +200,35 @@ def veda_topk_mask(layer: Layer, scores: torch.Tensor, k: Sequence[int], k_cap: 
                    mask: Optional[torch.Tensor] = None, stream=None):
     _check(_lib.veda_topk_mask(layer.ref, _ptr(scores), _host_i32(k), int(k_cap), _ptr(idx), _ptr(mask),
                                _stream(stream)))
+
+
+def veda_tile_scores_heads(layer: Layer, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden: int,
+                           out_dim: int, scale: float, scores: torch.Tensor, emb_ws: torch.Tensor,
+                           head_on: Optional[torch.Tensor], stream=None):
+    """veda_tile_scores for the (batch element, head) pairs with head_on != 0."""
+    _check(_lib.veda_tile_scores_heads(layer.ref, *[_ptr(t) for t in (dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k,
+                                                                        b2k)],
+                                       hidden, out_dim, float(scale), _ptr(scores), _ptr(emb_ws), _ptr(head_on),
+                                       _stream(stream)))
+
+
+def veda_topk_mask_heads(layer: Layer, scores: torch.Tensor, k: Sequence[int], k_cap: int, idx: torch.Tensor,
+                         mask: Optional[torch.Tensor], head_on: Optional[torch.Tensor], stream=None):
+    """veda_topk_mask for the (batch element, head) pairs with head_on != 0."""
+    _check(_lib.veda_topk_mask_heads(layer.ref, _ptr(scores), _host_i32(k), int(k_cap), _ptr(idx), _ptr(mask),
+                                     _ptr(head_on), _stream(stream)))
+
+
+def veda_score_cache_ws_bytes(layer: Layer) -> int:
+    return int(_lib.veda_score_cache_ws_bytes(layer.ref))
+
+
+def veda_score_cache_step(layer: Layer, dq, dk, dq_ref, dk_ref, tau: float, max_age: int, age: torch.Tensor,
+                          refresh: torch.Tensor, ws: torch.Tensor, stream=None):
+    """Temporal caching of tile scores: per (batch element, head), decide on
+    the device whether its cached mask is reused (refresh 0) or rebuilt."""
+    _check(_lib.veda_score_cache_step(layer.ref, _ptr(dq), _ptr(dk), _ptr(dq_ref), _ptr(dk_ref), float(tau),
+                                      int(max_age), _ptr(age), _ptr(refresh), _ptr(ws), _stream(stream)))
 
 
 def veda_tile_scores_topk(layer: Layer, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden: int, out_dim: int,

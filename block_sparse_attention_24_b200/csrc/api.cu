@@ -230,6 +230,14 @@ int veda_tile_scores(const veda_layer* L, const float* dq, const float* dk, cons
                      const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
                      const float* b2k, int32_t hidden, int32_t out_dim, float scale, float* scores, float* emb_ws,
                      cudaStream_t stream) {
+  return veda_tile_scores_heads(L, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, scale, scores,
+                                emb_ws, nullptr, stream);
+}
+
+int veda_tile_scores_heads(const veda_layer* L, const float* dq, const float* dk, const float* w1q, const float* b1q,
+                           const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
+                           const float* b2k, int32_t hidden, int32_t out_dim, float scale, float* scores,
+                           float* emb_ws, const int32_t* head_on, cudaStream_t stream) {
   veda::LayerGeom g;
   VEDA_TRY(build_geom(L, &g));
   const void* ptrs[] = {dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, scores, emb_ws};
@@ -239,13 +247,19 @@ int veda_tile_scores(const veda_layer* L, const float* dq, const float* dk, cons
     return fail(VEDA_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 4 in [4, 256]", hidden);
   if (out_dim < 4 || out_dim > 128 || out_dim % 4)
     return fail(VEDA_ERR_UNSUPPORTED, "out_dim=%d must be a multiple of 4 in [4, 128]", out_dim);
+  if (head_on) VEDA_TRY(check_ptr(head_on, "head_on"));
   return after_launch(veda::launch_tile_scores(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim,
-                                               scale, scores, emb_ws, stream),
+                                               scale, scores, emb_ws, stream, head_on),
                       "veda_tile_scores");
 }
 
 int veda_topk_mask(const veda_layer* L, const float* scores, const int32_t* k, int32_t k_cap, int32_t* idx,
                    uint8_t* mask, cudaStream_t stream) {
+  return veda_topk_mask_heads(L, scores, k, k_cap, idx, mask, nullptr, stream);
+}
+
+int veda_topk_mask_heads(const veda_layer* L, const float* scores, const int32_t* k, int32_t k_cap, int32_t* idx,
+                         uint8_t* mask, const int32_t* head_on, cudaStream_t stream) {
   veda::LayerGeom g;
   VEDA_TRY(build_geom(L, &g));
   VEDA_TRY(check_ptr(scores, "scores"));
@@ -258,7 +272,27 @@ int veda_topk_mask(const veda_layer* L, const float* scores, const int32_t* k, i
       return fail(VEDA_ERR_INVALID_ARG, "head %d: k=%d outside [1, min(nt=%d, k_cap=%d)]", h, k[h], g.h[h].nt, k_cap);
     g.h[h].k = k[h];
   }
-  return after_launch(veda::launch_topk(g, scores, k_cap, idx, mask, stream), "veda_topk_mask");
+  if (head_on) VEDA_TRY(check_ptr(head_on, "head_on"));
+  return after_launch(veda::launch_topk(g, scores, k_cap, idx, mask, stream, head_on), "veda_topk_mask");
+}
+
+size_t veda_score_cache_ws_bytes(const veda_layer* L) {
+  veda::LayerGeom g;
+  if (build_geom(L, &g) != VEDA_OK) return 0;
+  return veda::score_cache_ws_bytes(g);
+}
+
+int veda_score_cache_step(const veda_layer* L, const float* dq, const float* dk, float* dq_ref, float* dk_ref,
+                          float tau, int32_t max_age, int32_t* age, int32_t* refresh, void* ws, cudaStream_t stream) {
+  veda::LayerGeom g;
+  VEDA_TRY(build_geom(L, &g));
+  const void* ptrs[] = {dq, dk, dq_ref, dk_ref, age, refresh, ws};
+  const char* names[] = {"dq", "dk", "dq_ref", "dk_ref", "age", "refresh", "ws"};
+  for (int i = 0; i < 7; ++i) VEDA_TRY(check_ptr(ptrs[i], names[i]));
+  if (!(tau >= 0.f) || tau != tau) return fail(VEDA_ERR_INVALID_ARG, "tau=%g must be >= 0", (double)tau);
+  if (max_age < 1) return fail(VEDA_ERR_INVALID_ARG, "max_age=%d must be >= 1", max_age);
+  return after_launch(veda::launch_score_cache(g, dq, dk, dq_ref, dk_ref, tau, max_age, age, refresh, ws, stream),
+                      "veda_score_cache_step");
 }
 
 int veda_tile_scores_topk(const veda_layer* L, const float* dq, const float* dk, const float* w1q, const float* b1q,

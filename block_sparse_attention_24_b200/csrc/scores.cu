@@ -31,7 +31,9 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
                                                   const float* __restrict__ b2q, const float* __restrict__ w1k,
                                                   const float* __restrict__ b1k, const float* __restrict__ w2k,
                                                   const float* __restrict__ b2k, int hidden, int out_dim,
-                                                  float* __restrict__ emb) {
+                                                  float* __restrict__ emb, const int32_t* __restrict__ head_on) {
+  // head_on (may be NULL): per (batch element, head), 0 = keep the cached scores
+  if (head_on && !head_on[(blockIdx.z >> 1) * g.heads + blockIdx.y]) return;
   extern __shared__ float4 sm4[];
   float* sm = reinterpret_cast<float*>(sm4);
   const int din = 3 * g.d;
@@ -147,7 +149,9 @@ __global__ void __launch_bounds__(128) mlp_kernel(const __grid_constant__ LayerG
 
 // scores[b,h,i,j] = scale * q[i].k[j]; 64x64 output tile per CTA, 4x4 per thread.
 __global__ void __launch_bounds__(256) score_gemm_kernel(const __grid_constant__ LayerGeom g, const float* __restrict__ emb,
-                                                         int out_dim, float scale, float* __restrict__ scores) {
+                                                         int out_dim, float scale, float* __restrict__ scores,
+                                                         const int32_t* __restrict__ head_on) {
+  if (head_on && !head_on[blockIdx.z]) return;  // blockIdx.z = b * heads + h
   __shared__ float As[32][64 + 4];
   __shared__ float Bs[32][64 + 4];
   const int h = blockIdx.z % g.heads;
@@ -198,24 +202,28 @@ __global__ void __launch_bounds__(256) score_gemm_kernel(const __grid_constant__
 
 cudaError_t launch_mlp(const LayerGeom& g, const float* dq, const float* dk, const float* w1q, const float* b1q,
                        const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
-                       const float* b2k, int hidden, int out_dim, float* emb_ws, cudaStream_t s) {
+                       const float* b2k, int hidden, int out_dim, float* emb_ws, cudaStream_t s,
+                       const int32_t* head_on) {
   const size_t smem = (size_t)MLP_ROWS * (3 * g.d + hidden) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 g1((g.nt_cap + MLP_ROWS - 1) / MLP_ROWS, g.heads, g.B * 2);
-  mlp_kernel<<<g1, 128, smem, s>>>(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws);
+  mlp_kernel<<<g1, 128, smem, s>>>(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws,
+                                   head_on);
   return cudaGetLastError();
 }
 
 cudaError_t launch_tile_scores(const LayerGeom& g, const float* dq, const float* dk, const float* w1q,
                                const float* b1q, const float* w2q, const float* b2q, const float* w1k,
                                const float* b1k, const float* w2k, const float* b2k, int hidden, int out_dim,
-                               float scale, float* scores, float* emb_ws, cudaStream_t s) {
-  cudaError_t e = launch_mlp(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws, s);
+                               float scale, float* scores, float* emb_ws, cudaStream_t s,
+                               const int32_t* head_on) {
+  cudaError_t e = launch_mlp(g, dq, dk, w1q, b1q, w2q, b2q, w1k, b1k, w2k, b2k, hidden, out_dim, emb_ws, s,
+                             head_on);
   if (e != cudaSuccess) return e;
   const int nb = (g.nt_cap + 63) / 64;
   const dim3 g2(nb, nb, g.heads * g.B);
-  score_gemm_kernel<<<g2, 256, 0, s>>>(g, emb_ws, out_dim, scale, scores);
+  score_gemm_kernel<<<g2, 256, 0, s>>>(g, emb_ws, out_dim, scale, scores, head_on);
   return cudaGetLastError();
 }
 

@@ -108,7 +108,8 @@ __device__ __forceinline__ void warp_select_row(const uint32_t* keys, uint32_t* 
 
 __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_constant__ LayerGeom g,
                                                                const float* __restrict__ scores, int k_cap,
-                                                               int32_t* __restrict__ idx, uint8_t* __restrict__ mask) {
+                                                               int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
+                                                               const int32_t* __restrict__ head_on) {
   extern __shared__ uint32_t sm_u32[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   uint32_t* keys = sm_u32 + warp * (g.nt_cap + 256);
@@ -118,6 +119,8 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_cons
   if (row >= rows) return;
   const int a = (int)(row % g.nt_cap);
   const int h = (int)((row / g.nt_cap) % g.heads);
+  // head_on (may be NULL): per (batch element, head), 0 = keep the cached mask
+  if (head_on && !head_on[row / g.nt_cap]) return;
   const int nt = g.h[h].nt;
   const int k = g.h[h].k;
   int32_t* idx_row = idx + row * k_cap;
@@ -219,14 +222,14 @@ __global__ void __launch_bounds__(ST_THREADS) score_topk_kernel(const __grid_con
 }  // namespace
 
 cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int32_t* idx, uint8_t* mask,
-                        cudaStream_t s) {
+                        cudaStream_t s, const int32_t* head_on) {
   const size_t smem = (size_t)TOPK_WARPS * (g.nt_cap + 256) * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)g.B * g.heads * g.nt_cap;
   const long long blocks = (rows + TOPK_WARPS - 1) / TOPK_WARPS;
   if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
-  topk_kernel<<<(unsigned)blocks, TOPK_WARPS * 32, smem, s>>>(g, scores, k_cap, idx, mask);
+  topk_kernel<<<(unsigned)blocks, TOPK_WARPS * 32, smem, s>>>(g, scores, k_cap, idx, mask, head_on);
   return cudaGetLastError();
 }
 

@@ -428,7 +428,7 @@ cudaError_t launch_permute_pool(const LayerGeom& g, const void* x, void* xp, int
                                 cudaStream_t s);
 cudaError_t launch_mlp(const LayerGeom& g, const float* dq, const float* dk, const float* w1q, const float* b1q,
                        const float* w2q, const float* b2q, const float* w1k, const float* b1k, const float* w2k,
-                       const float* b2k, int hidden, int out_dim, float* emb_ws, cudaStream_t s);
+                       const float* b2k, int hidden, int out_dim, float* emb_ws, cudaStream_t s, const int32_t* head_on = nullptr);
 cudaError_t launch_score_topk(const LayerGeom& g, const float* emb_ws, int out_dim, float scale, int k_cap,
                               int32_t* idx, uint8_t* mask, float* scores, cudaStream_t s);
 size_t estimator_ws_floats_per_head(int nt_cap, int n_rows, int hidden, int out_dim, int din);
@@ -440,14 +440,17 @@ cudaError_t launch_output_sq_error(const LayerGeom& g, const void* a, const void
 cudaError_t launch_tile_scores(const LayerGeom& g, const float* dq, const float* dk, const float* w1q,
                                const float* b1q, const float* w2q, const float* b2q, const float* w1k,
                                const float* b1k, const float* w2k, const float* b2k, int hidden, int out_dim,
-                               float scale, float* scores, float* emb_ws, cudaStream_t s);
+                               float scale, float* scores, float* emb_ws, cudaStream_t s, const int32_t* head_on = nullptr);
 cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int32_t* idx, uint8_t* mask,
-                        cudaStream_t s);
+                        cudaStream_t s, const int32_t* head_on = nullptr);
 cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, int k_cap, float scale, void* op, float* lse,
                                cudaStream_t s, void* o_tokens = nullptr, bool tokens_in = false);
 // Token maps for Q, K (and V when non-NULL) of every distinct tiling; sets
 // each head's tmap. cudaErrorNotSupported past VEDA_MAX_TILINGS tilings.
+size_t score_cache_ws_bytes(const LayerGeom& g);
+cudaError_t launch_score_cache(const LayerGeom& g, const float* dq, const float* dk, float* dq_ref, float* dk_ref,
+                               float tau, int max_age, int32_t* age, int32_t* refresh, void* ws, cudaStream_t s);
 cudaError_t build_token_maps(LayerGeom& g, const void* q, const void* k, const void* v, TokenMaps* maps);
 cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int n_heads_sel, const int32_t* rows,
                               int n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,

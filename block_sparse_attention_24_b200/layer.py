@@ -13,13 +13,15 @@ from __future__ import annotations
 
 import math
 from dataclasses import dataclass
-from typing import Dict, List, Optional, Sequence
+from typing import Dict, List, Optional, Sequence, Tuple
 
 import torch
 
 from . import (Layer, veda_estimator_grad, veda_estimator_grad_ws_bytes, veda_full_attn_tilemax,
                veda_full_attn_tilemax_ws_bytes, veda_permute, veda_permute_trippool, veda_sparse_attn,
-               veda_sparse_attn_unpermute, veda_tile_scores,
+               veda_sparse_attn_unpermute, veda_score_cache_step, veda_score_cache_ws_bytes, veda_tile_scores,
+               veda_tile_scores_heads,
+               veda_topk_mask_heads,
                veda_tile_scores_ws_bytes, veda_topk_mask)
 
 
@@ -40,7 +42,11 @@ class VedaLayer:
               "unpermute", "tilemap_kl")
 
     def __init__(self, layer: Layer, keep: Optional[float], weights: Dict[str, torch.Tensor], score_scale: float,
-                 device, k: Optional[Sequence[int]] = None, maps: Optional[MapRequest] = None):
+                 device, k: Optional[Sequence[int]] = None, maps: Optional[MapRequest] = None,
+                 score_cache: Optional[Tuple[float, int]] = None):
+        """score_cache: (tau, max_age) to reuse each head's tile scores and
+        top-k mask across steps while its descriptors drift less than tau
+        (veda_score_cache_step); None rebuilds them every step."""
         self.L = layer
         self.device = device
         B, Hh, d = layer.B, layer.heads, layer.d
@@ -66,6 +72,9 @@ class VedaLayer:
         self.mask = torch.empty((B, Hh, nt_cap, nt_cap), dtype=torch.uint8, device=device)
         self.perm = torch.empty((Hh, n_cap), dtype=torch.int32, device=device)
         self.o = torch.empty((B, layer.N, Hh, d), **bf)
+        self.score_cache = None
+        if score_cache is not None:
+            self.enable_score_cache(*score_cache)
         self.maps = maps
         if maps is not None:
             nh = len(maps.heads)
@@ -74,6 +83,20 @@ class VedaLayer:
             self.kl_rows = torch.empty((nh, maps.n_rows), **f32)
             self.kl_out = torch.zeros(4, **f32)
             self.map_ws = torch.empty(veda_full_attn_tilemax_ws_bytes(layer, nh, maps.n_rows) // 4, **f32)
+
+    def enable_score_cache(self, tau: float, max_age: int):
+        """Start caching tile scores across steps (every head is rebuilt on
+        the next step); disable with `self.score_cache = None`."""
+        self.score_cache = (float(tau), int(max_age))
+        if not hasattr(self, "dq_ref"):
+            n = self.L.B * self.L.heads
+            self.dq_ref = torch.zeros_like(self.dq)
+            self.dk_ref = torch.zeros_like(self.dk)
+            self.cache_age = torch.full((n,), -1, dtype=torch.int32, device=self.device)
+            self.refresh = torch.ones((n,), dtype=torch.int32, device=self.device)
+            nbytes = veda_score_cache_ws_bytes(self.L)
+            self.cache_ws = torch.empty((nbytes + 15) // 16 * 4, dtype=torch.float32, device=self.device)
+        self.cache_age.fill_(-1)
 
     def effective_flops(self, idx_host=None) -> float:
         """4*d*sum of kept valid (query, key) token pairs over all heads, from
@@ -102,10 +125,20 @@ class VedaLayer:
         veda_permute_trippool(L, k, self.kp, self.dk, stream=stream)
         veda_permute(L, v, self.vp, stream=stream)
         w = self.w
-        veda_tile_scores(L, self.dq, self.dk, w["w1q"], w["b1q"], w["w2q"], w["b2q"], w["w1k"], w["b1k"], w["w2k"],
-                         w["b2k"], self.hidden, self.out_dim, self.score_scale, self.scores, self.emb_ws,
-                         stream=stream)
-        veda_topk_mask(L, self.scores, self.k, self.k_cap, self.idx, self.mask, stream=stream)
+        wts = (w["w1q"], w["b1q"], w["w2q"], w["b2q"], w["w1k"], w["b1k"], w["w2k"], w["b2k"])
+        if self.score_cache is None:
+            veda_tile_scores(L, self.dq, self.dk, *wts, self.hidden, self.out_dim, self.score_scale, self.scores,
+                             self.emb_ws, stream=stream)
+            veda_topk_mask(L, self.scores, self.k, self.k_cap, self.idx, self.mask, stream=stream)
+        else:
+            # per head on the device: reuse the cached scores and mask, or rebuild them
+            tau, max_age = self.score_cache
+            veda_score_cache_step(L, self.dq, self.dk, self.dq_ref, self.dk_ref, tau, max_age, self.cache_age,
+                                  self.refresh, self.cache_ws, stream=stream)
+            veda_tile_scores_heads(L, self.dq, self.dk, *wts, self.hidden, self.out_dim, self.score_scale,
+                                   self.scores, self.emb_ws, self.refresh, stream=stream)
+            veda_topk_mask_heads(L, self.scores, self.k, self.k_cap, self.idx, self.mask, self.refresh,
+                                 stream=stream)
 
     def attend(self, stream=None, out: Optional[torch.Tensor] = None):
         """Sparse attention with the output written in token order into `out`

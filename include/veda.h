@@ -201,6 +201,38 @@ int veda_sparse_attn_tokens(const veda_layer* L, const void* q, const void* k_in
                             const int32_t* idx, const int32_t* k, int32_t k_cap, float scale,
                             void* o, float* lse, cudaStream_t stream);
 
+/* Temporal caching of tile scores across diffusion steps (Veda summary 5
+ * names temporal caching of tile scores and adaptive sparsity across
+ * timesteps as future work; this rule is the library's reading). For every
+ * (batch element, head) bh: with D = the step's TripPool descriptors dq, dk
+ * and R = dq_ref, dk_ref (the descriptors of the step whose scores are
+ * cached), drift^2 = (|Dq-Rq|^2 + |Dk-Rk|^2) / (|Rq|^2 + |Rk|^2) over the
+ * head's valid tiles, summed in fp64 in a fixed order. refresh[bh] = 1 when
+ * age[bh] < 0 (never scored), age[bh] + 1 >= max_age, or drift^2 > tau^2;
+ * then age[bh] = 0 and R takes D; else refresh[bh] = 0 and age[bh] += 1.
+ * dq/dk/dq_ref/dk_ref: [B, heads, nt_cap, 3d] fp32 device; age, refresh:
+ * [B*heads] int32 device (initialise age to -1). tau >= 0, max_age >= 1
+ * (1 = refresh every step). ws: veda_score_cache_ws_bytes(L) bytes of device
+ * scratch (the per-chunk partial sums). Feed `refresh` to
+ * veda_tile_scores_heads and veda_topk_mask_heads: heads with 0 keep their
+ * scores, idx and mask. */
+size_t veda_score_cache_ws_bytes(const veda_layer* L);
+int veda_score_cache_step(const veda_layer* L, const float* dq, const float* dk, float* dq_ref, float* dk_ref,
+                          float tau, int32_t max_age, int32_t* age, int32_t* refresh, void* ws,
+                          cudaStream_t stream);
+
+/* veda_tile_scores and veda_topk_mask restricted to the (batch element,
+ * head) pairs with head_on[b*heads + h] != 0 (device int32 [B*heads], may be
+ * NULL = all): the other heads' scores, emb_ws rows, idx and mask are left as
+ * they are. */
+int veda_tile_scores_heads(const veda_layer* L, const float* dq, const float* dk,
+                           const float* w1q, const float* b1q, const float* w2q, const float* b2q,
+                           const float* w1k, const float* b1k, const float* w2k, const float* b2k,
+                           int32_t hidden, int32_t out_dim, float scale, float* scores,
+                           float* emb_ws, const int32_t* head_on, cudaStream_t stream);
+int veda_topk_mask_heads(const veda_layer* L, const float* scores, const int32_t* k, int32_t k_cap,
+                         int32_t* idx, uint8_t* mask, const int32_t* head_on, cudaStream_t stream);
+
 /* Oracle tile map and distillation loss (Veda summary 2.1, Target
  * Construction and Optimization; 2.3, Training Efficiency): for the selected
  * heads heads_sel[0..n_heads_sel) (HOST array) and query tiles

@@ -31,6 +31,7 @@ __all__ = [
     "mlp", "tile_scores", "topk_rows", "sparse_attention", "full_tilemap",
     "kl_rows", "recall", "k_from_keep", "effective_pairs",
     "gelu_grad", "estimator_loss", "estimator_grad", "tiling_errors",
+    "score_cache_step",
 ]
 
 
@@ -377,3 +378,40 @@ def tiling_errors(q, k, v, T, H, W, candidates, keep, scale):
         o = unpermute(op, perms, N)[0]
         errors[c] = ((o - full) ** 2).sum(axis=(0, 2))
     return errors
+
+
+# ---------------------------------------------------------------------------
+# 10. temporal caching of tile scores across diffusion steps (Veda summary 5
+#     names "temporal caching of tile scores" and adaptive sparsity across
+#     timesteps as future work; the rule is a [reading]: a head keeps the
+#     mask of its last refresh while its TripPool descriptors stay within a
+#     relative distance tau of that step's, for fewer than max_age steps)
+# ---------------------------------------------------------------------------
+
+def score_cache_step(dq, dk, dq_ref, dk_ref, nt, age, tau, max_age):
+    """One step of the cache rule for every (batch element, head).
+
+    dq, dk, dq_ref, dk_ref: [B, heads, nt_cap, 3d]; nt: tiles per head; age:
+    int array [B*heads], -1 = never scored. drift^2 = (|dq - dq_ref|^2 +
+    |dk - dk_ref|^2) / (|dq_ref|^2 + |dk_ref|^2) over the head's nt valid
+    tiles. Refresh when never scored, when age + 1 >= max_age, or when
+    drift^2 > tau^2 (compared as drift^2 numerator <= tau^2 * denominator).
+    Returns (refresh [B*heads] int, new age, new dq_ref, new dk_ref)."""
+    dq, dk = np.asarray(dq, np.float64), np.asarray(dk, np.float64)
+    dq_ref, dk_ref = np.array(dq_ref, np.float64), np.array(dk_ref, np.float64)
+    B, Hh = dq.shape[:2]
+    age = np.asarray(age, np.int64).copy()
+    refresh = np.zeros(B * Hh, np.int64)
+    for b in range(B):
+        for h in range(Hh):
+            i, n = b * Hh + h, int(nt[h])
+            num = ((dq[b, h, :n] - dq_ref[b, h, :n]) ** 2).sum() + ((dk[b, h, :n] - dk_ref[b, h, :n]) ** 2).sum()
+            den = (dq_ref[b, h, :n] ** 2).sum() + (dk_ref[b, h, :n] ** 2).sum()
+            fresh = age[i] < 0 or age[i] + 1 >= max_age or not (num <= tau * tau * den)
+            refresh[i] = int(fresh)
+            if fresh:
+                age[i] = 0
+                dq_ref[b, h, :n], dk_ref[b, h, :n] = dq[b, h, :n], dk[b, h, :n]
+            else:
+                age[i] += 1
+    return refresh, age, dq_ref, dk_ref

@@ -95,6 +95,11 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     rc = lib.veda_sparse_attn_tokens(L.ref, ctypes.c_void_p(0x1004), *[ctypes.c_void_p(0x1000)] * 2, None, None, 0,
                                      ctypes.c_float(0.1), ctypes.c_void_p(0x2000), None, None)
     assert rc == V.VEDA_ERR_INVALID_ARG and "q is not 16-byte aligned" in V.veda_last_error()
+    Q = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(7)]
+    rc = lib.veda_score_cache_step(L.ref, *Q[:4], ctypes.c_float(-0.1), 3, Q[4], Q[5], Q[6], None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "tau" in V.veda_last_error()
+    rc = lib.veda_score_cache_step(L.ref, *Q[:4], ctypes.c_float(0.1), 0, Q[4], Q[5], Q[6], None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "max_age" in V.veda_last_error()
     P = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(10)]
     rc = lib.veda_tile_scores_topk(L.ref, *P, 128, 64, ctypes.c_float(0.125), None, 4, ctypes.c_void_p(0x20000), None,
                                    None, ctypes.c_void_p(0x30000), None)

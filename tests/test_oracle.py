@@ -451,3 +451,51 @@ def test_tiling_errors_keep_all_and_designed_locality():
     assert e[0, 0] < 1e-20 and e[1, 0] > 1e-3                # head 0 wants frames
     assert e[1, 1] < 1e-20 and e[0, 1] > 1e-3                # head 1 wants x columns
     assert list(np.argmin(e, axis=0)) == [0, 1]
+
+
+def test_score_cache_rule_closed_forms():
+    """Temporal caching of tile scores (the [reading] of Veda summary 5): the
+    refresh rule on cases whose answer is fixed by arithmetic, not by
+    re-evaluating the oracle's formula."""
+    rng = np.random.default_rng(3)
+    B, Hh, nt_cap, din = 1, 3, 6, 12
+    nt = [6, 4, 5]
+    dq = rng.standard_normal((B, Hh, nt_cap, din))
+    dk = rng.standard_normal((B, Hh, nt_cap, din))
+    junk = np.full_like(dq, 99.0)
+    age = np.full(B * Hh, -1)
+    # first step: every head refreshes and takes the descriptors as reference
+    r, age, rq, rk = O.score_cache_step(dq, dk, junk, junk, nt, age, tau=0.3, max_age=4)
+    assert r.tolist() == [1, 1, 1] and age.tolist() == [0, 0, 0]
+    for h in range(Hh):
+        assert np.array_equal(rq[0, h, :nt[h]], dq[0, h, :nt[h]])
+    # unchanged descriptors: reused while age + 1 < max_age, then refreshed
+    seen = []
+    for _ in range(4):
+        r, age, rq, rk = O.score_cache_step(dq, dk, rq, rk, nt, age, tau=0.3, max_age=4)
+        seen.append(r.tolist())
+    assert seen == [[0, 0, 0], [0, 0, 0], [0, 0, 0], [1, 1, 1]]
+    # scaling Q and K by (1 + eps) moves them by exactly eps relative to the
+    # reference: 0.35 > tau refreshes (also when the drift would wrongly be
+    # measured against the new descriptors, 0.35/1.35 < 0.3); 0.25 keeps
+    age = np.zeros(B * Hh, int)
+    r, _, _, _ = O.score_cache_step(dq * 1.35, dk * 1.35, dq, dk, nt, age, tau=0.3, max_age=10)
+    assert r.tolist() == [1, 1, 1]
+    r, _, _, _ = O.score_cache_step(dq * 1.25, dk * 1.25, dq, dk, nt, age, tau=0.3, max_age=10)
+    assert r.tolist() == [0, 0, 0]
+    # a change in K alone counts; a change past nt (padding tiles) does not;
+    # heads are independent
+    dk2 = dk.copy()
+    dk2[0, 1, :nt[1]] *= 3.0
+    dq3 = dq.copy()
+    dq3[0, 2, nt[2]:] += 50.0
+    r, age2, rq2, _ = O.score_cache_step(dq3, dk2, dq, dk, nt, age, tau=0.3, max_age=10)
+    assert r.tolist() == [0, 1, 0] and age2.tolist() == [1, 0, 1]
+    assert np.array_equal(rq2[0, 0], dq[0, 0])
+    # max_age = 1 rebuilds every step; tau = 0 rebuilds on any change
+    r, _, _, _ = O.score_cache_step(dq, dk, dq, dk, nt, age, tau=0.3, max_age=1)
+    assert r.tolist() == [1, 1, 1]
+    dq4 = dq.copy()
+    dq4[0, 0, 0, 0] += 1e-9
+    r, _, _, _ = O.score_cache_step(dq4, dk, dq, dk, nt, age, tau=0.0, max_age=10)
+    assert r.tolist() == [1, 0, 0]
