@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import synth
-from block_sparse_attention_24_b200.layer import MapRequest, VedaLayer, device_weights
+from block_sparse_attention_24_b200.layer import VedaLayer, device_weights
+from tests.helpers import small_workloads
 from oracle import veda_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -24,9 +25,14 @@ def _layer(w, cache):
     return V, L, layer
 
 
-@pytest.mark.parametrize("idx", [0, 1])
-def test_score_cache_trajectory(idx):
-    w = synth.config(idx)
+CASES = {"cfg0": lambda: synth.config(0), "cfg1": lambda: synth.config(1),
+         "batch2": lambda: small_workloads()["batch2-d64-t128"],
+         "padded-d128-t128": lambda: small_workloads()["ragged-d128-t128"]}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_score_cache_trajectory(name):
+    w = CASES[name]()
     tau, max_age = 0.05, 3
     V, L, layer = _layer(w, (tau, max_age))
     q0, k0, v0 = synth.qkv(w, DEV)
