@@ -138,3 +138,16 @@ def test_empty_and_oversized_layers_rejected():
     assert e.value.code == V.VEDA_ERR_UNSUPPORTED and "exceeds" in str(e.value)
     with pytest.raises(V.VedaError):
         V.Layer(1, 129, 128, 4, 8, 8, 128, [(2, 8, 8)] * 129)
+
+
+def test_token_attention_tiling_limit():
+    """The token-order attention path keeps one tensor map per distinct tiling
+    and takes at most 8 of them: a layer with 9 is refused on the host,
+    before anything reaches the device."""
+    tilings = [(1, 8, 16), (1, 16, 8), (2, 8, 8), (2, 4, 16), (2, 16, 4), (4, 4, 8), (4, 8, 4), (8, 4, 4),
+               (8, 2, 8)]
+    L = V.Layer(1, len(tilings), 64, 16, 16, 16, 128, tilings)
+    lib = ctypes.CDLL(V.library_path())
+    p = ctypes.c_void_p(0x10000)
+    rc = lib.veda_sparse_attn_tokens(L.ref, p, p, p, None, None, 0, ctypes.c_float(0.125), p, None, None)
+    assert rc == V.VEDA_ERR_UNSUPPORTED and "8 distinct tilings" in V.veda_last_error()
