@@ -3,7 +3,8 @@
 // key/value tiles are loaded; here each loaded tile also serves both query
 // tiles of the CTA when both kept it).
 //
-// A CTA owns query tiles A = 2c and B = 2c+1 of one head. Every tile of the
+// A CTA owns two neighbouring query tiles A and B of one head (pair_stride:
+// along time for heads with p_t <= 2, else consecutive). Every tile of the
 // union of their kept lists is loaded by TMA exactly once, and S = Q K^T /
 // O += P V are issued only for the query tile(s) that kept it. Neighbouring
 // query tiles keep mostly the same key tiles (spatio-temporal locality), so
@@ -72,6 +73,20 @@ struct PairLayout {
   // dynamic shared memory for bitmaps of `words` 32-bit words each
   static constexpr int alloc(int words) { return OFF_BM + 8 * words + 1024; }
 };
+
+// Which two query tiles share a CTA: tiles a and a + S. For a head whose
+// tiles span at most two frames (p_t <= 2) neighbouring time slabs keep the
+// most key tiles in common, so S is the tiles per time slab; otherwise S = 1
+// (neighbours along W, or the next row). Measured on the benchmark layer's
+// kept lists, this cut the mean union of a pair from 1.27k to 1.21k.
+__host__ __device__ inline int pair_stride(const HeadGeom& hg) { return hg.pt <= 2 ? hg.tps : 1; }
+
+// CTAs of a head: ceil(n/2)*S pairs (n = nt/S tiles along the paired axis),
+// then one CTA per two padding tiles in [nt, nt_cap).
+__host__ __device__ inline int pair_ctas(const HeadGeom& hg, int nt_cap) {
+  const int S = pair_stride(hg), n = hg.nt / S;
+  return (n + 1) / 2 * S + (nt_cap - hg.nt + 1) / 2;
+}
 
 struct PairParams {
   int32_t k_cap;
@@ -311,8 +326,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const HeadGeom& hg = g.h[h];
   const int nt = hg.nt;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int qa = 2 * cp, qbt = 2 * cp + 1;  // the two query tiles
+  // the two query tiles (qbt >= nt: none), or two padding tiles to zero
+  int qa, qbt;
+  {
+    const int S = pair_stride(hg), n_axis = nt / S, n_pairs = (n_axis + 1) / 2 * S;
+    if (cp < n_pairs) {
+      const int j = cp / S, rr = cp - j * S;
+      qa = 2 * j * S + rr;
+      qbt = 2 * j + 1 < n_axis ? qa + S : nt;
+    } else {
+      qa = nt + 2 * (cp - n_pairs);
+      qbt = qa + 1;
+    }
+  }
   const long long rowA = (long long)bh * g.n_cap + (long long)qa * BM;
+  const long long rowB = (long long)bh * g.n_cap + (long long)qbt * BM;
 
   if (qa >= nt) {  // both query tiles are padding: zero output rows (none in token order)
     for (int i = threadIdx.x; prm.op && i < 2 * BM * D / 8; i += NUM_THREADS) {
@@ -623,7 +651,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive(p_full + r);
     }
     // epilogue: O / l -> bf16
-    const long long orow_i = rowA + (long long)r * BM + row;
+    const long long orow_i = (r ? rowB : rowA) + row;
     const bool in_range = a * BM + row < g.n_cap;
     if (kr == 0) {  // query tile beyond this head's tiles: zero rows (none in token order)
       if (in_range) {
@@ -696,7 +724,12 @@ cudaError_t launch_pair_t(const LayerGeom& g0, const void* qp, const void* kp, c
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((g.nt_cap + 1) / 2, g.heads, g.B);
+  int ctas = 1;
+  for (int h = 0; h < g.heads; ++h) {
+    const int c = pair_ctas(g.h[h], g.nt_cap);
+    ctas = c > ctas ? c : ctas;
+  }
+  const dim3 grid(ctas, g.heads, g.B);
   kern<<<grid, NUM_THREADS, smem, s>>>(g, maps, p);
   return cudaGetLastError();
 }
