@@ -1,14 +1,20 @@
 // Top-k key tiles per query tile (Veda summary 2.1 and 4: only the highest
 // scoring key tiles are kept).
 //
-// One warp per score row. The row is staged in shared memory as
-// order-preserving 32-bit keys (larger float -> larger key, -0.0 folded into
-// +0.0). A 4-pass, 8-bit radix select finds the exact k-th largest key T and
-// how many keys equal to T must be kept; a final pass in column order keeps
-// every key > T and the lowest-index keys == T, so exact ties go to the lower
-// tile index and the output list comes out ascending without a sort.
-// Histogram updates are warp-aggregated (__match_any_sync) shared atomics.
-// The same selection also runs inside the fused scores + top-k kernel.
+// One warp per score row; scores become order-preserving 32-bit keys (larger
+// float -> larger key, -0.0 folded into +0.0). The exact k-th largest key T
+// is found, then a final pass in column order keeps every key > T and the
+// lowest-index keys == T, so exact ties go to the lower tile index and the
+// output list comes out ascending without a sort.
+//
+// Rows of up to 2048 tiles (every layer of the pages' sizes) keep their keys
+// in registers, and T is built bit by bit from the top in 32 steps: a bit is
+// kept when at least k keys are >= T with it set. Each step is a compare and
+// count over the lane's keys and one warp reduction, with no shared memory and
+// no atomics. Longer rows are staged in shared memory and take a 4-pass,
+// 8-bit radix select whose histogram updates are warp-aggregated
+// (__match_any_sync) shared atomics; the same radix selection also runs inside
+// the fused scores + top-k kernel.
 #include "veda_internal.cuh"
 
 namespace veda {
@@ -106,7 +112,7 @@ __device__ __forceinline__ void warp_select_row(const uint32_t* keys, uint32_t* 
     for (int c = nt + lane; c < nt_cap; c += 32) mask_row[c] = 0;
 }
 
-__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_constant__ LayerGeom g,
+__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_radix_kernel(const __grid_constant__ LayerGeom g,
                                                                const float* __restrict__ scores, int k_cap,
                                                                int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
                                                                const int32_t* __restrict__ head_on) {
@@ -136,6 +142,93 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const __grid_cons
   __syncwarp();
 
   warp_select_row(keys, hist, nt, k, k_cap, g.nt_cap, idx_row, mask_row, lane);
+}
+
+// Register-resident selection: KPL keys per lane (column 32 i + lane in key
+// i; columns at or past nt hold key 0, which is below the key of every float,
+// so no candidate T >= 1 ever counts them).
+constexpr int BIS_WARPS = 8;
+
+template <int KPL>
+__global__ void __launch_bounds__(BIS_WARPS * 32) topk_bisect_kernel(const __grid_constant__ LayerGeom g,
+                                                                     const float* __restrict__ scores, int k_cap,
+                                                                     int32_t* __restrict__ idx,
+                                                                     uint8_t* __restrict__ mask,
+                                                                     const int32_t* __restrict__ head_on) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const long long rows = (long long)g.B * g.heads * g.nt_cap;
+  const long long row = (long long)blockIdx.x * BIS_WARPS + warp;
+  if (row >= rows) return;
+  const int a = (int)(row % g.nt_cap);
+  const int h = (int)((row / g.nt_cap) % g.heads);
+  if (head_on && !head_on[row / g.nt_cap]) return;
+  const int nt = g.h[h].nt;
+  const int k = g.h[h].k;
+  int32_t* idx_row = idx + row * k_cap;
+  uint8_t* mask_row = mask ? mask + row * g.nt_cap : nullptr;
+  if (a >= nt) {
+    for (int p = lane; p < k_cap; p += 32) idx_row[p] = -1;
+    if (mask_row)
+      for (int c = lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
+    return;
+  }
+  const float* srow = scores + row * g.nt_cap;
+  uint32_t key[KPL];
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int c = 32 * i + lane;
+    key[i] = c < nt ? order_key(__ldg(srow + c)) : 0u;
+  }
+  // T = the largest value with #(key >= T) >= k, i.e. the k-th largest key
+  // (the count only drops as T grows, so the top-down greedy choice is exact)
+  uint32_t T = 0u;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll
+    for (int i = 0; i < KPL; i += 4) {
+      c0 += key[i] >= cand;
+      c1 += key[i + 1] >= cand;
+      c2 += key[i + 2] >= cand;
+      c3 += key[i + 3] >= cand;
+    }
+    if (__reduce_add_sync(0xffffffffu, (unsigned)(c0 + c1 + c2 + c3)) >= (unsigned)k) T = cand;
+  }
+  int gt = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) gt += key[i] > T;
+  const int remaining = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);  // keys == T to keep, >= 1
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int base = 0, eq_seen = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    if (32 * i >= nt) break;
+    const int c = 32 * i + lane;
+    const bool in = c < nt;
+    const bool eq = in && key[i] == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_seen + __popc(eqm & lt_mask);
+    const bool sel = in && (key[i] > T || (eq && eq_rank < remaining));
+    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) idx_row[base + __popc(selm & lt_mask)] = c;
+    if (mask_row && in) mask_row[c] = sel ? 1 : 0;
+    base += __popc(selm);
+    eq_seen += __popc(eqm);
+  }
+  for (int p = k + lane; p < k_cap; p += 32) idx_row[p] = -1;
+  if (mask_row)
+    for (int c = nt + lane; c < g.nt_cap; c += 32) mask_row[c] = 0;
+}
+
+template <int KPL>
+cudaError_t launch_bisect(const LayerGeom& g, const float* scores, int k_cap, int32_t* idx, uint8_t* mask,
+                          cudaStream_t s, const int32_t* head_on) {
+  const long long rows = (long long)g.B * g.heads * g.nt_cap;
+  const long long blocks = (rows + BIS_WARPS - 1) / BIS_WARPS;
+  if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
+  topk_bisect_kernel<KPL><<<(unsigned)blocks, BIS_WARPS * 32, 0, s>>>(g, scores, k_cap, idx, mask, head_on);
+  return cudaGetLastError();
 }
 
 // Tile scores and top-k in one pass (Veda summary 2.1; the pages name
@@ -223,13 +316,27 @@ __global__ void __launch_bounds__(ST_THREADS) score_topk_kernel(const __grid_con
 
 cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int32_t* idx, uint8_t* mask,
                         cudaStream_t s, const int32_t* head_on) {
+  // register-resident keys: the smallest multiple of 8 keys per lane that
+  // holds a row
+  const int kpl = (g.nt_cap + 32 * 8 - 1) / (32 * 8) * 8;
+  switch (kpl) {
+    case 8: return launch_bisect<8>(g, scores, k_cap, idx, mask, s, head_on);
+    case 16: return launch_bisect<16>(g, scores, k_cap, idx, mask, s, head_on);
+    case 24: return launch_bisect<24>(g, scores, k_cap, idx, mask, s, head_on);
+    case 32: return launch_bisect<32>(g, scores, k_cap, idx, mask, s, head_on);
+    case 40: return launch_bisect<40>(g, scores, k_cap, idx, mask, s, head_on);
+    case 48: return launch_bisect<48>(g, scores, k_cap, idx, mask, s, head_on);
+    case 56: return launch_bisect<56>(g, scores, k_cap, idx, mask, s, head_on);
+    case 64: return launch_bisect<64>(g, scores, k_cap, idx, mask, s, head_on);
+    default: break;
+  }
   const size_t smem = (size_t)TOPK_WARPS * (g.nt_cap + 256) * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)g.B * g.heads * g.nt_cap;
   const long long blocks = (rows + TOPK_WARPS - 1) / TOPK_WARPS;
   if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
-  topk_kernel<<<(unsigned)blocks, TOPK_WARPS * 32, smem, s>>>(g, scores, k_cap, idx, mask, head_on);
+  topk_radix_kernel<<<(unsigned)blocks, TOPK_WARPS * 32, smem, s>>>(g, scores, k_cap, idx, mask, head_on);
   return cudaGetLastError();
 }
 

@@ -274,6 +274,18 @@ def test_topk_large_rows():
     _topk_case(w, s, oracle_k(w, lays))
 
 
+def test_topk_rows_past_register_path():
+    """Rows longer than 2048 tiles take the shared-memory radix selection."""
+    w = synth.custom("rows2112-d64-t64", 1, 2, 64, 33, 64, 64, 64, [(1, 8, 8), (1, 8, 8)], 0.1, 9)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    assert nt_cap == 2112
+    rng = np.random.default_rng(8)
+    s = (rng.standard_normal((1, w.heads, nt_cap, nt_cap)) * 3).astype(np.float32)
+    s = np.round(s * 64) / 64                              # frequent ties
+    _topk_case(w, s, oracle_k(w, lays))
+    _topk_case(w, s, [1, nt_cap])
+
+
 # --------------------------------------------------------- sparse attention
 
 def _attention_case(w, k_override=None, dense=False, random_lists=True, key_tile_gain=None, shuffle=False):
