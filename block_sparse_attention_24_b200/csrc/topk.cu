@@ -9,9 +9,9 @@
 //
 // Rows of up to 2048 tiles (every layer of the pages' sizes) keep their keys
 // in registers, and T is built bit by bit from the top in 32 steps: a bit is
-// kept when at least k keys are >= T with it set. Each step is a compare and
-// count over the lane's keys and one warp reduction, with no shared memory and
-// no atomics. Longer rows are staged in shared memory and take a 4-pass,
+// kept when at least k keys are >= T with it set. Each step counts the lane's
+// keys >= the candidate through an add-with-carry (two instructions per key)
+// and takes one warp reduction, with no shared memory and no atomics. Longer rows are staged in shared memory and take a 4-pass,
 // 8-bit radix select whose histogram updates are warp-aggregated
 // (__match_any_sync) shared atomics; the same radix selection also runs inside
 // the fused scores + top-k kernel.
@@ -149,6 +149,22 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_radix_kernel(const __gri
 // so no candidate T >= 1 ever counts them).
 constexpr int BIS_WARPS = 8;
 
+// #(keys >= cand) over one lane's keys, cand >= 1: key + (2^32 - cand)
+// carries out exactly when key >= cand, and the carry is added straight into
+// the count (two instructions per key).
+template <int KPL>
+__device__ __forceinline__ uint32_t count_ge(const uint32_t (&key)[KPL], uint32_t cand) {
+  const uint32_t neg = 0u - cand;
+  uint32_t c0 = 0u, c1 = 0u;
+#pragma unroll
+  for (int i = 0; i < KPL; i += 2) {
+    uint32_t t0, t1;
+    asm("add.cc.u32 %0, %2, %3;\n\taddc.u32 %1, %1, 0;" : "=r"(t0), "+r"(c0) : "r"(key[i]), "r"(neg));
+    asm("add.cc.u32 %0, %2, %3;\n\taddc.u32 %1, %1, 0;" : "=r"(t1), "+r"(c1) : "r"(key[i + 1]), "r"(neg));
+  }
+  return c0 + c1;
+}
+
 template <int KPL>
 __global__ void __launch_bounds__(BIS_WARPS * 32) topk_bisect_kernel(const __grid_constant__ LayerGeom g,
                                                                      const float* __restrict__ scores, int k_cap,
@@ -185,15 +201,7 @@ __global__ void __launch_bounds__(BIS_WARPS * 32) topk_bisect_kernel(const __gri
 #pragma unroll 1
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
-    int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
-#pragma unroll
-    for (int i = 0; i < KPL; i += 4) {
-      c0 += key[i] >= cand;
-      c1 += key[i + 1] >= cand;
-      c2 += key[i + 2] >= cand;
-      c3 += key[i + 3] >= cand;
-    }
-    if (__reduce_add_sync(0xffffffffu, (unsigned)(c0 + c1 + c2 + c3)) >= (unsigned)k) T = cand;
+    if (__reduce_add_sync(0xffffffffu, count_ge(key, cand)) >= (unsigned)k) T = cand;
   }
   int gt = 0;
 #pragma unroll
