@@ -35,7 +35,8 @@ __host__ __device__ inline int mlp_smem_floats(int din, int hidden) {
 // is read once per CTA (the eight warps share it through L1) and feeds
 // MLP_ROWS rows. Layer 1: each thread owns an MLP_RPT-row x 4-column
 // register tile of a 128-unit chunk (4*MLP_RPT FMAs per 16-byte weight
-// load), GELU'd and transposed into shared memory. Layer 2: 4 rows x 4
+// load, issued as packed fp32x2 FMAs, which round every lane like fmaf),
+// GELU'd and transposed into shared memory. Layer 2: 4 rows x 4
 // columns per thread over chunks of 64 outputs, so no lane idles at
 // out_dim = 64. (32 rows per CTA with 4 warps streamed each weight twice as
 // often per row and was L2-bound.)
@@ -103,11 +104,16 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const __grid_constant_
             const float4 x4 = *reinterpret_cast<const float4*>(xsT + i * MLP_ROWS + rg * MLP_RPT + 4 * q);
             xr[4 * q] = x4.x; xr[4 * q + 1] = x4.y; xr[4 * q + 2] = x4.z; xr[4 * q + 3] = x4.w;
           }
-          const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
+          const uint64_t w01 = f2(wv.x, wv.y), w23 = f2(wv.z, wv.w);
 #pragma unroll
-          for (int r = 0; r < MLP_RPT; ++r)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(xr[r], wr[e], acc[r][e]);
+          for (int r = 0; r < MLP_RPT; ++r) {
+            const uint64_t xx = f2(xr[r], xr[r]);
+            uint64_t a01 = f2(acc[r][0], acc[r][1]), a23 = f2(acc[r][2], acc[r][3]);
+            a01 = f2_fma(xx, w01, a01);
+            a23 = f2_fma(xx, w23, a23);
+            f2_split(a01, acc[r][0], acc[r][1]);
+            f2_split(a23, acc[r][2], acc[r][3]);
+          }
         }
       }
       if (alias) __syncthreads();  // every thread is done with the descriptors (single chunk)
