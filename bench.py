@@ -217,7 +217,8 @@ def run_ours(args, world, rank, local):
     elapsed = max_over_ranks(elapsed, device)
     V.veda_check_status(L)
     front_ms = statistics.mean(e["start"].elapsed_time(e["front"]) for e in ev)
-    attn_ms = statistics.mean(e["attn0"].elapsed_time(e["attn1"]) for e in ev)
+    attn_each = [e["attn0"].elapsed_time(e["attn1"]) for e in ev]
+    attn_ms = statistics.mean(attn_each)  # the roofline's average launch duration
     unperm_ms = statistics.mean(e["attn1"].elapsed_time(e["unpermute"]) for e in ev)
     tail_ms = statistics.mean(e["unpermute"].elapsed_time(e["end"]) for e in ev)
     clk.__exit__(None, None, None)
@@ -260,8 +261,10 @@ def run_ours(args, world, rank, local):
         "config": bench_config(w, world, round(1 - kept / allp, 4), int(layer.maps.n_rows)),
         "attn_ms": round(attn_ms, 3), "attn_tflops": round(attn_tflops, 1),
         "attn_frac_of_burst_peak": round(attn_tflops / burst, 4),
+        "attn_ms_median": round(statistics.median(attn_each), 3), "attn_ms_min": round(min(attn_each), 3),
         "dense_ms": round(dense_ms, 3), "speedup_vs_dense": round(dense_ms / attn_ms, 2),
         "layer_ms": round(front_ms + attn_ms + unperm_ms, 3),
+        "speedup_layer_vs_dense": round(dense_ms / (front_ms + attn_ms + unperm_ms), 2),
         "stage_ms": {**stage_ms, "front_end": round(front_ms, 3), "sparse_attn": round(attn_ms, 3),
                      "unpermute": round(unperm_ms, 3), "tilemap_kl": round(tail_ms, 3)},
         "estimator_grad_ms": grad_ms,
