@@ -74,17 +74,40 @@ __global__ void __launch_bounds__(256) permute_kernel(const __grid_constant__ La
 // Forward permutation fused with TripPool (Veda summary 2.1 and 2.2): the
 // CTA that moves a tile's rows also reduces them to the tile descriptor
 // [mean | max | min] per channel, so the permuted tensor is never read back.
-// Each thread keeps sum / max / min of its 8 channels over the valid rows it
-// moves; threads holding the same channels are combined with warp shuffles
-// and then across the 8 warps through shared memory in a fixed order.
+// Each valid row of the tile (one token's slice of this head: D bf16, a
+// 16-byte multiple) is copied into shared memory by cp.async.bulk on one
+// mbarrier, so a CTA keeps its whole tile in flight with few registers; the
+// padding rows are zeroed in shared memory; one bulk store writes the tile to
+// its contiguous permuted slots; the descriptor is reduced from shared
+// memory, 256 threads over channel pairs x row groups, combined in a fixed
+// order. (Holding the rows in registers took 61 registers a thread, 4 CTAs
+// per SM, and was 5% slower.)
+__device__ __forceinline__ void bulk_load_row(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_tile(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(smem_src)),
+               "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 template <int VPR>
 __global__ void __launch_bounds__(256) permute_pool_kernel(const __grid_constant__ LayerGeom g,
-                                                           const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                                           int32_t* __restrict__ perm, float* __restrict__ desc) {
+                                                                const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                                int32_t* __restrict__ perm, float* __restrict__ desc) {
   constexpr int D = VPR * 8;
-  __shared__ int s_off[128];
-  __shared__ int s_lt[128];
-  __shared__ float part[8][VPR][24];
+  constexpr uint32_t RB = D * 2;         // bytes per row
+  constexpr int NCP = D / 2;             // channel pairs
+  constexpr int NG = 256 / NCP;          // row groups
+  extern __shared__ __align__(128) uint8_t rows_sm[];  // [tile][D] bf16
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_abort;
+  __shared__ float part[NG][6][NCP];
   const int tid = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const HeadGeom& hg = g.h[h];
   const int tile = g.tile;
@@ -100,106 +123,83 @@ __global__ void __launch_bounds__(256) permute_pool_kernel(const __grid_constant
       for (int i = threadIdx.x; i < 3 * D; i += blockDim.x) out[i] = 0.f;
     return;
   }
-  const int slab = hg.ph * hg.pw;
-  if (threadIdx.x < tile) {
-    const int loc = threadIdx.x;
-    const int lt = loc / slab;
-    const int lr = loc - lt * slab;
-    const int ly = lr / hg.pw;
-    const int lx = lr - ly * hg.pw;
-    s_lt[loc] = lt;
-    s_off[loc] = (lt * g.H + ly) * g.W + lx;
-  }
+  const int nv = tile_len(hg, g.T, tid);  // the valid rows are a prefix of the tile
   const int tt = tid / hg.tps;
   const int rem = tid - tt * hg.tps;
   const int th = rem / hg.nwt;
   const int tw = rem - th * hg.nwt;
   const int t0 = tt * hg.pt;
   const int n0 = (t0 * g.H + th * hg.ph) * g.W + tw * hg.pw;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    s_abort = 0;
+    fence_mbar_init();
+    mbar_expect_tx(&bar, (uint32_t)nv * RB);
+  }
+  __syncthreads();  // the expected bytes are registered before any copy can complete
+  if (threadIdx.x < tile) {
+    const int loc = threadIdx.x;
+    const int slab = hg.ph * hg.pw;
+    const int lt = loc / slab;
+    const int lr = loc - lt * slab;
+    const int ly = lr / hg.pw;
+    const int lx = lr - ly * hg.pw;
+    const int n = n0 + (lt * g.H + ly) * g.W + lx;
+    if (loc < nv) {
+      bulk_load_row(rows_sm + loc * RB, src + (((long long)b * N + n) * g.heads + h) * VPR, RB, &bar);
+    } else {
+      uint4* z = reinterpret_cast<uint4*>(rows_sm + loc * RB);
+#pragma unroll
+      for (int e = 0; e < VPR; ++e) z[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (perm && b == 0) perm[(long long)h * g.n_cap + tid * tile + loc] = loc < nv ? n : -1;
+  }
+  if (!mbar_wait(&bar, 0, &s_abort, g.dev_status)) {
+    mbar_wait_drain(&bar, 0, VEDA_WAIT_LIMIT_NS);  // let the copies into this CTA's memory land
+    return;
+  }
+  fence_proxy_async_smem();  // the zeroed padding rows, before the bulk store reads them
   __syncthreads();
-
-  float sum[8], mx[8], mn[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    sum[e] = 0.f;
-    mx[e] = -INFINITY;
-    mn[e] = INFINITY;
+  if (threadIdx.x == 0) bulk_store_tile(dst + slot0 * VPR, rows_sm, (uint32_t)tile * RB);
+  const int cp = threadIdx.x % NCP, grp = threadIdx.x / NCP;
+  float s0 = 0.f, s1 = 0.f, hi0 = -INFINITY, hi1 = -INFINITY, lo0 = INFINITY, lo1 = INFINITY;
+  for (int r = grp; r < nv; r += NG) {
+    const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(rows_sm + r * RB)[cp]);
+    s0 += f.x;
+    s1 += f.y;
+    hi0 = fmaxf(hi0, f.x);
+    hi1 = fmaxf(hi1, f.y);
+    lo0 = fminf(lo0, f.x);
+    lo1 = fminf(lo1, f.y);
   }
-  // all of a thread's rows are loaded before any is stored or reduced, so
-  // each thread keeps up to RPT independent 16-byte loads in flight
-  constexpr int RPP = 256 / VPR;  // rows per pass
-  constexpr int RPT = 128 / RPP;  // rows per thread for a 128-token tile
-  const int v = threadIdx.x % VPR;
-  const int r0 = threadIdx.x / VPR;
-  uint4 val[RPT];
-  bool ok[RPT];
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    const int r = r0 + i * RPP;
-    ok[i] = r < tile && t0 + s_lt[r < tile ? r : 0] < g.T;
-    val[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (ok[i]) {
-      const long long orow = ((long long)b * N + n0 + s_off[r]) * g.heads + h;
-      val[i] = __ldg(src + orow * VPR + v);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    const int r = r0 + i * RPP;
-    if (r < tile) {
-      dst[(slot0 + r) * VPR + v] = val[i];
-      if (perm && b == 0 && v == 0) perm[(long long)h * g.n_cap + tid * tile + r] = ok[i] ? n0 + s_off[r] : -1;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    if (ok[i]) {
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&val[i]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(p2[e]);
-        sum[2 * e] += f.x;
-        sum[2 * e + 1] += f.y;
-        mx[2 * e] = fmaxf(mx[2 * e], f.x);
-        mx[2 * e + 1] = fmaxf(mx[2 * e + 1], f.y);
-        mn[2 * e] = fminf(mn[2 * e], f.x);
-        mn[2 * e + 1] = fminf(mn[2 * e + 1], f.y);
-      }
-    }
-  }
-  // lanes v, v+VPR, ... of a warp hold the same channels
-#pragma unroll
-  for (int off = VPR; off < 32; off <<= 1) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      sum[e] += __shfl_xor_sync(0xffffffffu, sum[e], off);
-      mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
-      mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], off));
-    }
-  }
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (lane < VPR) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      part[warp][lane][e] = sum[e];
-      part[warp][lane][8 + e] = mx[e];
-      part[warp][lane][16 + e] = mn[e];
-    }
-  }
+  part[grp][0][cp] = s0;
+  part[grp][1][cp] = s1;
+  part[grp][2][cp] = hi0;
+  part[grp][3][cp] = hi1;
+  part[grp][4][cp] = lo0;
+  part[grp][5][cp] = lo1;
   __syncthreads();
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x, cv = c / 8, ce = c % 8;
-    float S = part[0][cv][ce], M = part[0][cv][8 + ce], m = part[0][cv][16 + ce];
+  if (threadIdx.x < NCP) {
+    float S0 = part[0][0][cp], S1 = part[0][1][cp], H0 = part[0][2][cp], H1 = part[0][3][cp];
+    float L0 = part[0][4][cp], L1 = part[0][5][cp];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) {  // fixed order: bit-reproducible
-      S += part[w][cv][ce];
-      M = fmaxf(M, part[w][cv][8 + ce]);
-      m = fminf(m, part[w][cv][16 + ce]);
+    for (int q = 1; q < NG; ++q) {  // fixed order: bit-reproducible
+      S0 += part[q][0][cp];
+      S1 += part[q][1][cp];
+      H0 = fmaxf(H0, part[q][2][cp]);
+      H1 = fmaxf(H1, part[q][3][cp]);
+      L0 = fminf(L0, part[q][4][cp]);
+      L1 = fminf(L1, part[q][5][cp]);
     }
-    out[c] = S / (float)tile_len(hg, g.T, tid);
-    out[D + c] = M;
-    out[2 * D + c] = m;
+    const float cnt = (float)nv;
+    out[2 * cp] = S0 / cnt;
+    out[2 * cp + 1] = S1 / cnt;
+    out[D + 2 * cp] = H0;
+    out[D + 2 * cp + 1] = H1;
+    out[2 * D + 2 * cp] = L0;
+    out[2 * D + 2 * cp + 1] = L1;
   }
+  if (threadIdx.x == 0) bulk_wait_read_all();  // the tile stays in shared memory until the store has read it
 }
 
 }  // namespace
@@ -218,10 +218,11 @@ cudaError_t launch_permute(const LayerGeom& g, const void* x, void* xp, int32_t*
 cudaError_t launch_permute_pool(const LayerGeom& g, const void* x, void* xp, int32_t* perm, float* desc,
                                 cudaStream_t s) {
   const dim3 grid(g.nt_cap, g.heads, g.B);
+  const size_t smem = (size_t)g.tile * g.d * 2;
   if (g.d == 128)
-    permute_pool_kernel<16><<<grid, 256, 0, s>>>(g, (const uint4*)x, (uint4*)xp, perm, desc);
+    permute_pool_kernel<16><<<grid, 256, smem, s>>>(g, (const uint4*)x, (uint4*)xp, perm, desc);
   else
-    permute_pool_kernel<8><<<grid, 256, 0, s>>>(g, (const uint4*)x, (uint4*)xp, perm, desc);
+    permute_pool_kernel<8><<<grid, 256, smem, s>>>(g, (const uint4*)x, (uint4*)xp, perm, desc);
   return cudaGetLastError();
 }
 
