@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -91,7 +92,8 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # raw samples go to $VEDA_CLOCKS_DIR (default: the system temp directory)
+        self.path = os.path.join(os.environ.get("VEDA_CLOCKS_DIR") or tempfile.gettempdir(), f"clocks_rank{index}.csv")
 
     def __enter__(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
