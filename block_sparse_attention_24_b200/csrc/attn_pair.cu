@@ -4,7 +4,8 @@
 // tiles of the CTA when both kept it).
 //
 // A CTA owns two neighbouring query tiles A and B of one head (pair_stride:
-// along time for heads with p_t <= 2, else consecutive). Every tile of the
+// along time for heads with p_t <= 2 and an even number of time slabs, else
+// consecutive). Every tile of the
 // union of their kept lists is loaded by TMA exactly once, and S = Q K^T /
 // O += P V are issued only for the query tile(s) that kept it. Neighbouring
 // query tiles keep mostly the same key tiles (spatio-temporal locality), so
@@ -79,7 +80,12 @@ struct PairLayout {
 // most key tiles in common, so S is the tiles per time slab; otherwise S = 1
 // (neighbours along W, or the next row). Measured on the benchmark layer's
 // kept lists, this cut the mean union of a pair from 1.27k to 1.21k.
-__host__ __device__ inline int pair_stride(const HeadGeom& hg) { return hg.pt <= 2 ? hg.tps : 1; }
+// Along time only when the time slabs pair up exactly: with an odd count the
+// last slab's tps tiles would run alone, where consecutive pairing leaves at
+// most one tile alone.
+__host__ __device__ inline int pair_stride(const HeadGeom& hg) {
+  return hg.pt <= 2 && (hg.nt / hg.tps) % 2 == 0 ? hg.tps : 1;
+}
 
 // CTAs of a head: ceil(n/2)*S pairs (n = nt/S tiles along the paired axis),
 // then one CTA per two padding tiles in [nt, nt_cap).
