@@ -5,13 +5,16 @@ A step is one pass of the whole hot path over one synthetic layer (the
 128-token tiles, 10% of key tiles kept = 90% sparsity):
   permute Q,K,V -> TripPool Q,K -> MLP tile scores -> top-k mask
   -> tile-skipping sparse attention -> inverse permute
-  -> full-attention tile map + row-wise KL on 2 heads x 120 query tiles.
+  -> full-attention tile map + row-wise KL on 2 heads x 120 query tiles
+  -> recall of the top-k mask against the tile map's own top-k on those rows.
 
 `value` is effective attention TFLOP/s over the whole step (4*d*kept valid
 token pairs / step time); the attention kernel alone, the library's dense
 path at sparsity 0 and the roofline of the attention kernel are reported
 beside it. `--impl reference` times the fp64 CPU oracle on a bounded sample
-of the same workload.
+of the same workload. Beside the step the line carries the same layer at 95%
+sparsity (attention, dense-path speedup, recall) and the attention kernel on
+the 24,576-token (64-token tiles) and 80,640-token layers.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -39,7 +42,7 @@ import synth  # noqa: E402
 METRIC = "block-sparse attn ms/layer & effective TFLOP/s at 90% sparsity vs dense path"
 UNIT = "TFLOP/s"
 MAP_ROWS = 120          # query tiles per tile-map head (10% of 1200: sparse supervision)
-KERNELS_PER_STEP = 11   # 2 permute+TripPool, permute V, MLP + score GEMM, top-k, attention (output in token order), map sweep + finish, KL rows, KL mean
+KERNELS_PER_STEP = 13   # 2 permute+TripPool, permute V, MLP + score GEMM, top-k, attention (output in token order), map sweep + finish, KL rows, KL mean, recall rows + mean
 
 
 # ------------------------------------------------------------------ ranks
@@ -164,17 +167,18 @@ def build_layer(w, device, seed_offset=0):
     return V, L, layer, (q, k, v)
 
 
-def kept_pairs(L, layer):
+def kept_pairs(L, layer, idx=None, k=None):
     """Kept valid (query, key) token pairs and all valid pairs, from the
-    top-k lists and the tile lengths."""
-    idx = layer.idx.cpu()
+    top-k lists (default: the layer's own) and the tile lengths."""
+    idx = (layer.idx if idx is None else idx).cpu()
+    k = layer.k if k is None else k
     kept = allp = 0
     for h in range(L.heads):
         pt, ph, pw = L.tilings[h]
         tps = (L.H // ph) * (L.W // pw)
         lens = torch.tensor([min(pt, L.T - (t // tps) * pt) * ph * pw for t in range(L.nt[h])], dtype=torch.int64)
         for b in range(L.B):
-            rows = idx[b, h, :L.nt[h], :layer.k[h]].long()
+            rows = idx[b, h, :L.nt[h], :k[h]].long()
             kept += int((lens * lens[rows].sum(dim=1)).sum())
             allp += int(lens.sum()) ** 2
     return kept, allp
@@ -249,34 +253,47 @@ def run_ours(args, world, rank, local):
 
     burst, sustained, hbm, src = measured_peaks()
     attn_tflops = eff_flops / (attn_ms / 1e3) / 1e12
+    layer_ms = front_ms + attn_ms + unperm_ms
     step_ms = elapsed / args.steps * 1e3
     value = world * eff_flops / (elapsed / args.steps) / 1e12
-    traffic = load_traffic()
-    hbm_stages = frontend_bandwidth(L, layer, stage_ms, unperm_ms, hbm)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, layer, L, budget_s=args.cpu_seconds)
+    traffic = load_traffic()
+    hbm_stages = frontend_bandwidth(L, layer, stage_ms, unperm_ms, hbm)
+    alu_stages = frontend_compute(L, layer, stage_ms, clocks.get("sm_mhz"))
+    recall90 = layer_recall(layer)
+    map_rows = int(layer.maps.n_rows)
+    sp95 = run_keep(V, L, layer, q, k, v, 0.05, dense_ms, burst, stream)
+    del layer, q, k, v
+    torch.cuda.empty_cache()
+    others = {} if args.no_other_layers else other_layers(device, burst, stream)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": bench_config(w, world, round(1 - kept / allp, 4), int(layer.maps.n_rows)),
+        "config": bench_config(w, world, round(1 - kept / allp, 4), map_rows),
         "attn_ms": round(attn_ms, 3), "attn_tflops": round(attn_tflops, 1),
         "attn_frac_of_burst_peak": round(attn_tflops / burst, 4),
         "attn_ms_median": round(statistics.median(attn_each), 3), "attn_ms_min": round(min(attn_each), 3),
         "dense_ms": round(dense_ms, 3), "speedup_vs_dense": round(dense_ms / attn_ms, 2),
-        "layer_ms": round(front_ms + attn_ms + unperm_ms, 3),
-        "speedup_layer_vs_dense": round(dense_ms / (front_ms + attn_ms + unperm_ms), 2),
+        "layer_ms": round(layer_ms, 3),
+        "speedup_layer_vs_dense": round(dense_ms / layer_ms, 2),
         "stage_ms": {**stage_ms, "front_end": round(front_ms, 3), "sparse_attn": round(attn_ms, 3),
                      "unpermute": round(unperm_ms, 3), "tilemap_kl": round(tail_ms, 3)},
         "estimator_grad_ms": grad_ms,
         "score_cache": cache_ms,
-        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": sustained, "unit": UNIT,
-                     "frac": round(attn_tflops / sustained, 4), "traffic": traffic,
+        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": burst, "unit": UNIT,
+                     "frac": round(attn_tflops / burst, 4), "traffic": traffic,
                      "kernel": "sparse_attn_pair_kernel<128>",
                      "kernel_source_sha256_16": kernel_source_hash(),
-                     "peak_kind": f"bf16 dense sustained ({src}); burst {burst}"},
+                     "peak_kind": f"bf16 dense burst ({src}): the kernel is timed launch by launch",
+                     "frac_of_sustained": round(attn_tflops / sustained, 4)},
+        "recall": recall90,
+        "sparsity_95": sp95,
+        "other_layers": others,
         "hbm_stages": hbm_stages,
+        "alu_stages": alu_stages,
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
@@ -287,6 +304,119 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+def layer_recall(layer) -> dict:
+    """Recall of the step's top-k mask against the tile map's own top-k on
+    the map rows (computed inside the step by the recall kernels)."""
+    r = layer.recall.cpu().tolist()
+    m = layer.maps
+    return {"mean": round(r[-1], 4), "per_head": {str(h): round(x, 4) for h, x in zip(m.heads, r[:-1])},
+            "rows_per_head": int(m.n_rows), "k": [layer.k[h] for h in m.heads],
+            "note": "untrained (Xavier-initialised) estimator: reported, not targeted"}
+
+
+def time_launches(fn, stream, reps, warm=2, flush=None):
+    """Mean and min of `reps` launches of fn, each bracketed by CUDA events on
+    `stream` (optionally writing `flush`, a buffer larger than L2, between
+    launches)."""
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.add_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ts]
+    return statistics.mean(ms), min(ms)
+
+
+def run_keep(V, L, layer, q, k, v, keep, dense_ms, burst, stream, reps=10) -> dict:
+    """The same layer at another keep fraction: top-k of the step's scores at
+    that k, the attention kernel (output in token order) timed launch by
+    launch, its speedup over the same dense-path time, and the recall of that
+    mask against the step's tile map."""
+    from block_sparse_attention_24_b200.layer import k_from_keep
+    kk = [k_from_keep(keep, nt) for nt in L.nt]
+    k_cap = max(kk)
+    idx = torch.empty((L.B, L.heads, L.nt_cap, k_cap), dtype=torch.int32, device=layer.device)
+    V.veda_topk_mask(L, layer.scores, kk, k_cap, idx, None)
+    hits = torch.empty_like(layer.recall_hits)
+    rec = torch.empty_like(layer.recall)
+    layer.map_recall(idx, kk, k_cap, hits, rec)
+    out = torch.empty_like(layer.o)
+    fn = lambda: V.veda_sparse_attn_unpermute(L, layer.qp, layer.kp, layer.vp, idx, kk, k_cap, layer.attn_scale, out)
+    mean_ms, min_ms = time_launches(fn, stream, reps)
+    V.veda_check_status(L)
+    kept, allp = kept_pairs(L, layer, idx, kk)
+    tf = 4.0 * L.d * kept / (mean_ms / 1e3) / 1e12
+    r = rec.cpu().tolist()
+    return {"keep": keep, "k": kk[0] if len(set(kk)) == 1 else kk, "sparsity": round(1 - kept / allp, 4),
+            "attn_ms": round(mean_ms, 3), "attn_ms_min": round(min_ms, 3), "attn_tflops": round(tf, 1),
+            "attn_frac_of_burst_peak": round(tf / burst, 4), "speedup_vs_dense": round(dense_ms / mean_ms, 2),
+            "recall": {"mean": round(r[-1], 4), "per_head": {str(h): round(x, 4) for h, x in zip(layer.maps.heads, r[:-1])}}}
+
+
+def other_layers(device, burst, stream) -> dict:
+    """The attention kernel on the 24,576-token layer (12 heads, 64-token
+    tiles, 80% sparsity) and the 80,640-token layer (40 heads, T padded per
+    tiling, 90% sparsity): each launch timed on its own after an L2 flush,
+    and the same kernel's dense path."""
+    out = {}
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)   # 256 MB > L2
+    for cfg in (1, 2):
+        w = synth.config(cfg)
+        V, L, layer, (q, k, v) = build_layer(w, device)
+        layer.forward(q, k, v)
+        torch.cuda.synchronize()
+        kept, allp = kept_pairs(L, layer)
+        mean_ms, min_ms = time_launches(lambda: layer.attend(stream), stream, 10, flush=flush)
+        dout = torch.empty_like(layer.op)
+        dense_ms, _ = time_launches(lambda: layer.dense(dout), stream, 2, warm=1, flush=flush)
+        V.veda_check_status(L)
+        tf = 4.0 * L.d * kept / (mean_ms / 1e3) / 1e12
+        out[w.name] = {"tokens": w.N, "heads": w.heads, "tile": w.tile, "sparsity": round(1 - kept / allp, 4),
+                       "attn_ms": round(mean_ms, 3), "attn_ms_min": round(min_ms, 3), "attn_tflops": round(tf, 1),
+                       "attn_frac_of_burst_peak": round(tf / burst, 4), "dense_ms": round(dense_ms, 3),
+                       "dense_tflops": round(4.0 * L.d * allp / (dense_ms / 1e3) / 1e12, 1),
+                       "speedup_vs_dense": round(dense_ms / mean_ms, 2), "l2": "flushed before every launch",
+                       "recall": round(float(layer.recall[-1]), 4) if layer.maps is not None else None}
+        del layer, q, k, v, dout
+        torch.cuda.empty_cache()
+    return out
+
+
+def frontend_compute(L, layer, stage_ms, sm_mhz) -> dict:
+    """The compute-bound front-end stages against bounds derived from the SM
+    count and the sampled SM clock: the MLP and score GEMM against the fp32
+    FMA rate (148 SMs x 128 FMA lanes x 2 flop per clock), the top-k against
+    the instruction issue rate (148 SMs x 4 schedulers x 1 warp instruction
+    per clock) for its counting loop (2 integer instructions per key and
+    bisection step, 32 steps, keys padded to the register layout)."""
+    if not sm_mhz:
+        return {}
+    f = sm_mhz * 1e6
+    d3, hid, out_dim = 3 * L.d, layer.hidden, layer.out_dim
+    nts = [L.nt[h] for h in range(L.heads)] * L.B
+    mlp = sum(2 * nt * 2 * (d3 * hid + hid * out_dim) for nt in nts)
+    gemm = sum(2 * nt * nt * out_dim for nt in nts)
+    ffma_peak = 148 * 128 * 2 * f
+    kpl = (L.nt_cap + 255) // 256 * 8
+    rows = L.B * L.heads * L.nt_cap
+    issue = rows * 32 * 2 * kpl
+    issue_peak = 148 * 4 * f
+    ts, tk = stage_ms["tile_scores"] / 1e3, stage_ms["topk"] / 1e3
+    return {"clock_mhz": sm_mhz,
+            "tile_scores": {"bound": "fp32 fma", "flop": mlp + gemm, "ms": stage_ms["tile_scores"],
+                            "tflops": round((mlp + gemm) / ts / 1e12, 2), "peak_tflops": round(ffma_peak / 1e12, 1),
+                            "frac": round((mlp + gemm) / ts / ffma_peak, 3)},
+            "topk": {"bound": "issue", "warp_instructions": issue, "ms": stage_ms["topk"],
+                     "frac": round(issue / tk / issue_peak, 3)}}
 
 
 def stage_breakdown(V, L, layer, q, k, v, stream):
@@ -503,7 +633,7 @@ def cpu_baseline(w, layer, L, budget_s):
     idx = layer.idx[0, h].cpu().numpy()
     flops, secs, tiles = oracle_attention_sample(w, qp, kp, vp, idx, layer.k[h], lens, budget_s)
     return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"fp64 NumPy sparse attention, head {h}, {tiles} random query tiles of 1200 "
+            "sample": f"fp64 NumPy sparse attention, head {h}, {tiles} random query tiles of {L.nt[h]} "
                       f"({secs:.1f} s); the front end is not included"}
 
 
@@ -624,6 +754,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-layers", action="store_true", help="skip the 24,576- and 80,640-token attention timings")
     ap.add_argument("--sweep", action="store_true", help="head-group token/sparsity sweep instead of the step")
     args = ap.parse_args()
     if args.warmup < 3:

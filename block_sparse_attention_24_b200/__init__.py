@@ -27,7 +27,7 @@ VEDA_ERR_BAD_INDEX = -5
 
 EXPORTED = ("veda_layout", "veda_permute", "veda_trippool", "veda_permute_trippool", "veda_tile_scores", "veda_tile_scores_ws_bytes",
             "veda_tile_scores_noalloc",
-            "veda_topk_mask", "veda_tile_scores_topk", "veda_tile_scores_heads", "veda_topk_mask_heads", "veda_score_cache_step", "veda_score_cache_ws_bytes", "veda_sparse_attn", "veda_sparse_attn_unpermute", "veda_sparse_attn_tokens", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes", "veda_tilemap_kl",
+            "veda_topk_mask", "veda_tile_scores_topk", "veda_tile_scores_heads", "veda_topk_mask_heads", "veda_score_cache_step", "veda_score_cache_ws_bytes", "veda_sparse_attn", "veda_sparse_attn_unpermute", "veda_sparse_attn_tokens", "veda_full_attn_tilemax", "veda_full_attn_tilemax_ws_bytes", "veda_tilemap_kl", "veda_tilemap_recall",
             "veda_check_status",
             "veda_estimator_grad", "veda_estimator_grad_ws_bytes", "veda_output_sq_error", "veda_selftest_wait_timeout", "veda_last_error")
 
@@ -83,6 +83,7 @@ _lib.veda_full_attn_tilemax.argtypes = [_LP, _P, _P, _P, _I, _P, _I, _F, _P, _P,
 _lib.veda_full_attn_tilemax_ws_bytes.argtypes = [_LP, _I, _I]
 _lib.veda_tilemap_kl.argtypes = [_LP, _P, _I, _P, _I, _P, _P, _P, _P, _P]
 _lib.veda_full_attn_tilemax_ws_bytes.restype = ctypes.c_size_t
+_lib.veda_tilemap_recall.argtypes = [_LP, _P, _I, _P, _I, _P, _P, _P, _I, _P, _P, _P, _P]
 _lib.veda_estimator_grad.argtypes = [_LP] + [_P] * 10 + [_I, _I, _F, _P, _I, _P, _I, _P] + [_P] * 8 + [_P, _P, _P]
 _lib.veda_estimator_grad_ws_bytes.argtypes = [_LP, _I, _I, _I, _I]
 _lib.veda_estimator_grad_ws_bytes.restype = ctypes.c_size_t
@@ -93,7 +94,7 @@ _lib.veda_last_error.restype = ctypes.c_char_p
 for _name in EXPORTED:
     getattr(_lib, _name)
     if _name not in ("veda_last_error", "veda_tile_scores_ws_bytes", "veda_estimator_grad_ws_bytes",
-                     "veda_full_attn_tilemax_ws_bytes"):
+                     "veda_full_attn_tilemax_ws_bytes", "veda_score_cache_ws_bytes"):
         getattr(_lib, _name).restype = ctypes.c_int
 
 
@@ -278,6 +279,16 @@ def veda_tilemap_kl(layer: Layer, heads_sel: Sequence[int], qtile_rows: Optional
                     stream=None):
     _check(_lib.veda_tilemap_kl(layer.ref, _host_i32(heads_sel), len(heads_sel), _ptr(qtile_rows), int(n_rows),
                                 _ptr(tilemap), _ptr(scores), _ptr(kl_rows), _ptr(kl_out), _stream(stream)))
+
+
+def veda_tilemap_recall(layer: Layer, heads_sel: Sequence[int], qtile_rows: Optional[torch.Tensor], n_rows: int,
+                        tilemap: torch.Tensor, idx: torch.Tensor, k: Sequence[int], k_cap: int, hits: torch.Tensor,
+                        recall: torch.Tensor, map_idx: Optional[torch.Tensor] = None, stream=None):
+    """hits [n_heads_sel, n_rows] int32, recall [n_heads_sel + 1] fp32 (per
+    head, then their mean); map_idx (optional) the map's own top-k lists."""
+    _check(_lib.veda_tilemap_recall(layer.ref, _host_i32(heads_sel), len(heads_sel), _ptr(qtile_rows), int(n_rows),
+                                    _ptr(tilemap), _ptr(idx), _host_i32(k), int(k_cap), _ptr(hits), _ptr(map_idx),
+                                    _ptr(recall), _stream(stream)))
 
 
 def veda_full_attn_tilemax_ws_bytes(layer: Layer, n_heads_sel: int, n_rows: int) -> int:

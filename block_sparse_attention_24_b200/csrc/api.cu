@@ -446,6 +446,41 @@ int veda_tilemap_kl(const veda_layer* L, const int32_t* heads_sel, int32_t n_hea
                       "veda_tilemap_kl");
 }
 
+int veda_tilemap_recall(const veda_layer* L, const int32_t* heads_sel, int32_t n_heads_sel,
+                        const int32_t* qtile_rows, int32_t n_rows, const float* tilemap, const int32_t* idx,
+                        const int32_t* k, int32_t k_cap, int32_t* hits, int32_t* map_idx, float* recall,
+                        cudaStream_t stream) {
+  veda::LayerGeom g;
+  VEDA_TRY(build_geom(L, &g));
+  if (g.B != 1) return fail(VEDA_ERR_UNSUPPORTED, "recall: only B == 1 layers are accepted");
+  VEDA_TRY(check_ptr(tilemap, "tilemap"));
+  VEDA_TRY(check_ptr(idx, "idx"));
+  VEDA_TRY(check_ptr(hits, "hits"));
+  VEDA_TRY(check_ptr(recall, "recall"));
+  if (map_idx) VEDA_TRY(check_ptr(map_idx, "map_idx"));
+  if (qtile_rows) VEDA_TRY(check_ptr(qtile_rows, "qtile_rows"));
+  if (!heads_sel || n_heads_sel < 1 || n_heads_sel > VEDA_MAX_HEADS)
+    return fail(VEDA_ERR_INVALID_ARG, "heads_sel must list 1..%d heads", VEDA_MAX_HEADS);
+  if (n_rows < 1) return fail(VEDA_ERR_INVALID_ARG, "n_rows=%d must be >= 1", n_rows);
+  if (!k) return fail(VEDA_ERR_INVALID_ARG, "k is NULL");
+  if (k_cap < 1 || k_cap > VEDA_MAX_NT) return fail(VEDA_ERR_INVALID_ARG, "k_cap=%d outside [1, %d]", k_cap, VEDA_MAX_NT);
+  for (int h = 0; h < g.heads; ++h) {
+    if (k[h] < 1 || k[h] > g.h[h].nt || k[h] > k_cap)
+      return fail(VEDA_ERR_INVALID_ARG, "head %d: k=%d outside [1, min(nt=%d, k_cap=%d)]", h, k[h], g.h[h].nt, k_cap);
+    g.h[h].k = k[h];
+  }
+  for (int s = 0; s < n_heads_sel; ++s) {
+    if (heads_sel[s] < 0 || heads_sel[s] >= g.heads)
+      return fail(VEDA_ERR_INVALID_ARG, "heads_sel[%d]=%d outside [0, %d)", s, heads_sel[s], g.heads);
+    if (!qtile_rows && n_rows > g.h[heads_sel[s]].nt)
+      return fail(VEDA_ERR_INVALID_ARG, "n_rows=%d exceeds the %d tiles of head %d", n_rows,
+                  g.h[heads_sel[s]].nt, heads_sel[s]);
+  }
+  return after_launch(veda::launch_recall(g, heads_sel, n_heads_sel, qtile_rows, n_rows, tilemap, idx, k_cap, hits,
+                                          map_idx, recall, stream),
+                      "veda_tilemap_recall");
+}
+
 size_t veda_estimator_grad_ws_bytes(const veda_layer* L, int32_t n_heads_sel, int32_t n_rows, int32_t hidden,
                                     int32_t out_dim) {
   veda::LayerGeom g;

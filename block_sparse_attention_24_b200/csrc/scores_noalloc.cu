@@ -33,7 +33,11 @@ void* g_scratch_ptr[VEDA_NOALLOC_MAX_DEVICES] = {};
 
 // Device address of this device's copy of the array. In host code the array's
 // name only stands for it; the address comes from cudaGetSymbolAddress, called
-// once per device with that device current (first call on each device).
+// once per device with that device current (first call on each device). With
+// lazy module loading that first lookup is also what loads this module on the
+// device, and with it reserves the array. The address is cached for the life
+// of the process: a cudaDeviceReset would leave it stale, so the entry point
+// is documented as unsupported across one.
 cudaError_t scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

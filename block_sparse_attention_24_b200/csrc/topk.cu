@@ -320,6 +320,112 @@ __global__ void __launch_bounds__(ST_THREADS) score_topk_kernel(const __grid_con
   }
 }
 
+// Recall of the predicted top-k lists against the tile map's own top-k
+// (Veda summary 2.1, Target Construction: the max-pooled full-attention map
+// is the target the estimator is aligned to). One warp per (selected head,
+// sampled query tile): the map row is ranked exactly as a score row is ranked
+// here (order keys, the head's k, exact ties to the lower tile index) into a
+// list in shared memory; the hits are the tiles held both by that list and
+// by the predicted list of the same query tile, counted over two kept-tile
+// bitmaps (set semantics, so a repeated predicted entry counts once).
+struct RecallParams {
+  int32_t heads_sel[VEDA_MAX_HEADS];
+  const int32_t* rows;    // [n_sel, n_rows] query tiles, or NULL: 0..n_rows-1
+  const float* tilemap;   // [n_sel, n_rows, nt_cap]
+  const int32_t* idx;     // predicted lists [B = 1, heads, nt_cap, k_cap]
+  int32_t* map_idx;       // [n_sel, n_rows, k_cap] or NULL
+  int32_t* hits;          // [n_sel, n_rows]
+  float* recall;          // [n_sel + 1]
+  int32_t n_sel, n_rows, k_cap, warps;
+};
+
+// 32-bit words of one warp's shared area: order keys, radix histogram, the
+// map's selected list, and two kept-tile bitmaps.
+__host__ __device__ inline int recall_warp_words(int nt_cap, int k_cap) {
+  return nt_cap + 256 + k_cap + 2 * ((nt_cap + 31) / 32);
+}
+
+__global__ void __launch_bounds__(128) recall_rows_kernel(const __grid_constant__ LayerGeom g,
+                                                          const __grid_constant__ RecallParams prm) {
+  extern __shared__ uint32_t sm_u32[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int words = (g.nt_cap + 31) / 32;
+  uint32_t* keys = sm_u32 + warp * recall_warp_words(g.nt_cap, prm.k_cap);
+  uint32_t* hist = keys + g.nt_cap;
+  int32_t* sel = reinterpret_cast<int32_t*>(hist + 256);
+  uint32_t* bm_map = reinterpret_cast<uint32_t*>(sel + prm.k_cap);
+  uint32_t* bm_pred = bm_map + words;
+  const long long row = (long long)blockIdx.x * prm.warps + warp;
+  if (warp >= prm.warps || row >= (long long)prm.n_sel * prm.n_rows) return;
+  const int s = (int)(row / prm.n_rows), r = (int)(row % prm.n_rows);
+  const int h = prm.heads_sel[s];
+  const int nt = g.h[h].nt, k = g.h[h].k;
+  const int a = prm.rows ? __ldg(prm.rows + row) : r;
+  int32_t* mrow = prm.map_idx ? prm.map_idx + row * prm.k_cap : nullptr;
+  if (a < 0 || a >= nt) {  // not a query tile of this head: no hits, empty list
+    if (lane == 0) {
+      prm.hits[row] = 0;
+      report(g.dev_status, VEDA_ERR_BAD_INDEX);
+    }
+    if (mrow)
+      for (int p = lane; p < prm.k_cap; p += 32) mrow[p] = -1;
+    return;
+  }
+  const float* M = prm.tilemap + row * g.nt_cap;
+  for (int c = lane; c < nt; c += 32) keys[c] = order_key(__ldg(M + c));
+  for (int w = lane; w < words; w += 32) bm_map[w] = bm_pred[w] = 0u;
+  __syncwarp();
+  warp_select_row(keys, hist, nt, k, prm.k_cap, g.nt_cap, sel, nullptr, lane);
+  __syncwarp();
+  const int32_t* pred = prm.idx + ((long long)h * g.nt_cap + a) * prm.k_cap;
+  bool bad = false;
+  for (int p = lane; p < k; p += 32) {
+    const int t = sel[p];
+    atomicOr(bm_map + (t >> 5), 1u << (t & 31));
+    const int u = __ldg(pred + p);
+    if (u >= 0 && u < nt) atomicOr(bm_pred + (u >> 5), 1u << (u & 31));
+    else bad = true;
+  }
+  __syncwarp();
+  if (__any_sync(0xffffffffu, bad) && lane == 0) report(g.dev_status, VEDA_ERR_BAD_INDEX);
+  unsigned c = 0;
+  for (int w = lane; w < words; w += 32) c += __popc(bm_map[w] & bm_pred[w]);
+  c = __reduce_add_sync(0xffffffffu, c);
+  if (lane == 0) prm.hits[row] = (int32_t)c;
+  if (mrow)
+    for (int p = lane; p < prm.k_cap; p += 32) mrow[p] = sel[p];
+}
+
+// recall[s] = (sum of head s's hits) / (n_rows * k_h); recall[n_sel] = the
+// mean over the selected heads, in head order. Hit sums are integers, so the
+// result does not depend on the order of the additions.
+__global__ void __launch_bounds__(256) recall_mean_kernel(const __grid_constant__ LayerGeom g,
+                                                          const __grid_constant__ RecallParams prm) {
+  __shared__ unsigned long long part[256];
+  __shared__ double per_head[VEDA_MAX_HEADS];
+  for (int s = 0; s < prm.n_sel; ++s) {
+    unsigned long long c = 0;
+    for (int r = threadIdx.x; r < prm.n_rows; r += 256) c += (unsigned long long)prm.hits[(long long)s * prm.n_rows + r];
+    part[threadIdx.x] = c;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+      if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      const double v = (double)part[0] / ((double)prm.n_rows * g.h[prm.heads_sel[s]].k);
+      per_head[s] = v;
+      prm.recall[s] = (float)v;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    double m = 0.0;
+    for (int s = 0; s < prm.n_sel; ++s) m += per_head[s];
+    prm.recall[prm.n_sel] = (float)(m / prm.n_sel);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const LayerGeom& g, const float* scores, int k_cap, int32_t* idx, uint8_t* mask,
@@ -364,6 +470,36 @@ cudaError_t launch_score_topk(const LayerGeom& g, const float* emb_ws, int out_d
   if (e != cudaSuccess) return e;
   const dim3 grid((g.nt_cap + R - 1) / R, g.heads, g.B);
   score_topk_kernel<<<grid, ST_THREADS, smem, s>>>(g, emb_ws, out_dim, scale, R, k_cap, idx, mask, scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_recall(const LayerGeom& g, const int32_t* heads_sel, int n_sel, const int32_t* rows, int n_rows,
+                          const float* tilemap, const int32_t* idx, int k_cap, int32_t* hits, int32_t* map_idx,
+                          float* recall, cudaStream_t s) {
+  RecallParams prm;
+  for (int i = 0; i < VEDA_MAX_HEADS; ++i) prm.heads_sel[i] = i < n_sel ? heads_sel[i] : 0;
+  prm.rows = rows;
+  prm.tilemap = tilemap;
+  prm.idx = idx;
+  prm.map_idx = map_idx;
+  prm.hits = hits;
+  prm.recall = recall;
+  prm.n_sel = n_sel;
+  prm.n_rows = n_rows;
+  prm.k_cap = k_cap;
+  const size_t per_warp = (size_t)recall_warp_words(g.nt_cap, k_cap) * sizeof(uint32_t);
+  int warps = (int)((200 * 1024) / per_warp);
+  warps = warps > 4 ? 4 : warps;
+  if (warps < 1) return cudaErrorInvalidValue;
+  prm.warps = warps;
+  const size_t smem = (size_t)warps * per_warp;
+  cudaError_t e = cudaFuncSetAttribute(recall_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long total = (long long)n_sel * n_rows;
+  recall_rows_kernel<<<(unsigned)((total + warps - 1) / warps), 128, smem, s>>>(g, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  recall_mean_kernel<<<1, 256, 0, s>>>(g, prm);
   return cudaGetLastError();
 }
 

@@ -455,6 +455,9 @@ cudaError_t build_token_maps(LayerGeom& g, const void* q, const void* k, const v
 cudaError_t launch_tilemap_kl(const LayerGeom& g, const int32_t* heads_sel, int n_heads_sel, const int32_t* rows,
                               int n_rows, const float* tilemap, const float* scores, float* kl_rows, float* kl_out,
                               cudaStream_t s);
+cudaError_t launch_recall(const LayerGeom& g, const int32_t* heads_sel, int n_sel, const int32_t* rows, int n_rows,
+                          const float* tilemap, const int32_t* idx, int k_cap, int32_t* hits, int32_t* map_idx,
+                          float* recall, cudaStream_t s);
 size_t tilemax_ws_bytes(int n_heads_sel, int n_rows, int tile, int nt_cap);
 cudaError_t launch_tilemax(const LayerGeom& g, const void* qp, const void* kp, const int32_t* heads_sel,
                            int n_heads_sel, const int32_t* rows, int n_rows, float scale, float* tilemap, float* lse,

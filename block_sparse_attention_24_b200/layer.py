@@ -4,7 +4,8 @@ order, over buffers allocated once.
     permute + TripPool (Q, K), permute (V) -> tile scores -> top-k mask
       -> tile-skipping sparse attention -> inverse permute
     (+ distillation rows: full-attention tile map on selected heads and query
-       tiles, row-wise KL against the predicted scores)
+       tiles, row-wise KL against the predicted scores, recall of the
+       predicted mask against the map's own top-k)
 
 Only marshalling and buffer management live here; every step is a libveda
 kernel launch.
@@ -20,7 +21,7 @@ import torch
 from . import (Layer, veda_estimator_grad, veda_estimator_grad_ws_bytes, veda_full_attn_tilemax,
                veda_full_attn_tilemax_ws_bytes, veda_permute, veda_permute_trippool, veda_sparse_attn,
                veda_sparse_attn_unpermute, veda_score_cache_step, veda_score_cache_ws_bytes, veda_tile_scores,
-               veda_tile_scores_heads,
+               veda_tile_scores_heads, veda_tilemap_recall,
                veda_topk_mask_heads,
                veda_tile_scores_ws_bytes, veda_topk_mask)
 
@@ -83,6 +84,8 @@ class VedaLayer:
             self.kl_rows = torch.empty((nh, maps.n_rows), **f32)
             self.kl_out = torch.zeros(4, **f32)
             self.map_ws = torch.empty(veda_full_attn_tilemax_ws_bytes(layer, nh, maps.n_rows) // 4, **f32)
+            self.recall_hits = torch.empty((nh, maps.n_rows), dtype=torch.int32, device=device)
+            self.recall = torch.zeros(nh + 1, **f32)   # per map head, then their mean
 
     def enable_score_cache(self, tau: float, max_age: int):
         """Start caching tile scores across steps (every head is rebuilt on
@@ -159,6 +162,14 @@ class VedaLayer:
         m = self.maps
         veda_full_attn_tilemax(self.L, self.qp, self.kp, m.heads, m.rows, m.n_rows, self.attn_scale, self.tilemap,
                                self.map_lse, self.scores, self.kl_rows, self.kl_out, ws=self.map_ws, stream=stream)
+        self.map_recall(self.idx, self.k, self.k_cap, self.recall_hits, self.recall, stream=stream)
+
+    def map_recall(self, idx, k, k_cap, hits, recall, map_idx=None, stream=None):
+        """Recall of predicted key-tile lists `idx` (k per head) against the
+        top-k of this step's tile-map rows (call after distill's map)."""
+        m = self.maps
+        veda_tilemap_recall(self.L, m.heads, m.rows, m.n_rows, self.tilemap, idx, k, k_cap, hits, recall,
+                            map_idx=map_idx, stream=stream)
 
     def estimator_grad(self, stream=None):
         """Weight gradient of the distillation loss on this step's tile-map

@@ -129,9 +129,16 @@ size_t veda_tile_scores_ws_bytes(const veda_layer* L, int32_t out_dim);
  * (16 MiB, held by every GPU that loads the library until the process
  * exits); a layer needing more (veda_tile_scores_ws_bytes > 16 MiB) is
  * rejected with VEDA_ERR_UNSUPPORTED. The first call on each device looks up
- * that device's copy of the array (make it before any stream capture). All
- * calls share the array: calls whose kernels may overlap on the GPU race and
- * must be serialised by the caller. Allocates nothing. */
+ * that device's copy of the array with cudaGetSymbolAddress; with CUDA's
+ * lazy module loading this is also when the driver loads the library's
+ * device code on that device and so reserves the array, which can fail
+ * (VEDA_ERR_CUDA) if the device has no room left. Make that first call once
+ * per device at initialisation, before any stream capture and outside
+ * per-frame loops; later calls reserve nothing. The looked-up address is kept
+ * for the life of the process, so the call is not supported across a
+ * cudaDeviceReset. All calls share the array: calls whose kernels may overlap
+ * on the GPU race and must be serialised by the caller. The call itself
+ * allocates no device memory. */
 int veda_tile_scores_noalloc(const veda_layer* L, const float* dq, const float* dk,
                              const float* w1q, const float* b1q, const float* w2q, const float* b2q,
                              const float* w1k, const float* b1k, const float* w2k, const float* b2k,
@@ -270,6 +277,32 @@ int veda_full_attn_tilemax(const veda_layer* L, const void* qp, const void* kp,
 int veda_tilemap_kl(const veda_layer* L, const int32_t* heads_sel, int32_t n_heads_sel,
                     const int32_t* qtile_rows, int32_t n_rows, const float* tilemap,
                     const float* scores, float* kl_rows, float* kl_out, cudaStream_t stream);
+
+/* Recall of the predicted key-tile lists against the tile map (Veda summary
+ * 2.1, Target Construction: the max-pooled full-attention map is the target
+ * the estimator is aligned to; Veda summary 1 and 4 judge the kept tiles by
+ * how much of the attention they hold). For the selected heads heads_sel
+ * (HOST array) and query tiles qtile_rows [n_heads_sel, n_rows] (DEVICE
+ * int32; NULL = tiles 0..n_rows-1), with tilemap the output of
+ * veda_full_attn_tilemax for the same heads and rows:
+ *   map top-k: the k[h] tiles of the map row ranked exactly as
+ *              veda_topk_mask ranks a score row (fp32 value, exact ties and
+ *              -0.0/+0.0 to the lower tile index);
+ *   hits[s, r] = |set(idx[0, h, a, 0..k[h])) & map top-k|, a = the query tile;
+ *   recall[s]  = sum_r hits[s, r] / (n_rows * k[h]);
+ *   recall[n_heads_sel] = the mean of recall[0..n_heads_sel) in head order.
+ * idx: the predicted lists [1, heads, nt_cap, k_cap] int32 (veda_topk_mask
+ * output); k: HOST array [heads] as given to veda_topk_mask. hits
+ * [n_heads_sel, n_rows] int32 and recall [n_heads_sel + 1] fp32 are DEVICE
+ * outputs; map_idx (may be NULL) [n_heads_sel, n_rows, k_cap] int32 receives
+ * the map's own top-k lists (ascending, -1 padded). A query tile outside its
+ * head or a predicted entry outside [0, nt_h) is reported as
+ * VEDA_ERR_BAD_INDEX in dev_status (that row then counts the valid entries
+ * only). Only B == 1 layers are accepted. */
+int veda_tilemap_recall(const veda_layer* L, const int32_t* heads_sel, int32_t n_heads_sel,
+                        const int32_t* qtile_rows, int32_t n_rows, const float* tilemap, const int32_t* idx,
+                        const int32_t* k, int32_t k_cap, int32_t* hits, int32_t* map_idx, float* recall,
+                        cudaStream_t stream);
 
 /* Estimator training (Veda summary 2.1, Optimization: the head-specific
  * projections are trained with the row-wise KL against the tile map, with

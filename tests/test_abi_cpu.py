@@ -116,6 +116,17 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     assert rc == V.VEDA_ERR_INVALID_ARG and "heads_sel" in V.veda_last_error()
     rc = lib.veda_tilemap_kl(L.ref, sel, 1, None, 1, ctypes.c_void_p(0x1000), None, None, None, None)
     assert rc == V.VEDA_ERR_INVALID_ARG and "scores" in V.veda_last_error()
+    k_ok = (ctypes.c_int32 * 2)(2, 1)
+    rc = lib.veda_tilemap_recall(L.ref, sel, 1, None, 1, *[ctypes.c_void_p(0x1000)] * 2, k_ok, 8,
+                                 *[ctypes.c_void_p(0x1000)] * 3, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "heads_sel" in V.veda_last_error()
+    sel0 = (ctypes.c_int32 * 1)(0)
+    rc = lib.veda_tilemap_recall(L.ref, sel0, 1, None, 1, *[ctypes.c_void_p(0x1000)] * 2, k, 8,
+                                 *[ctypes.c_void_p(0x1000)] * 3, None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "k=5" in V.veda_last_error()
+    rc = lib.veda_tilemap_recall(L.ref, sel0, 1, None, 1, *[ctypes.c_void_p(0x1000)] * 2, k_ok, 8,
+                                 None, None, ctypes.c_void_p(0x1000), None)
+    assert rc == V.VEDA_ERR_INVALID_ARG and "hits" in V.veda_last_error()
     rc = lib.veda_check_status(None, None)
     assert rc == V.VEDA_ERR_INVALID_ARG
 

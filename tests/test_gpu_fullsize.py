@@ -124,6 +124,15 @@ def test_full_layer_sampled(name):
         s_gpu = layer.scores[0, h, :nt, :nt].cpu().numpy()
         kl = O.kl_rows(M, s_gpu[rows_all[s, pick]])
         np.testing.assert_allclose(klr[s, pick], kl, rtol=1e-3, atol=1e-5)
+        # recall of the predicted mask against the map's top-k, every sampled
+        # row: exact against the oracle's recall on the GPU's map rows
+        kk = layer.k[h]
+        mask = layer.mask[0, h, rows_all[s], :nt].cpu().numpy().astype(bool)
+        hits = layer.recall_hits[s].cpu().numpy()
+        for r in range(m.n_rows):
+            assert hits[r] == round(O.recall(mask[r:r + 1], tm[s, r:r + 1, :nt].astype(np.float32), kk) * kk)
+        assert float(layer.recall[s]) == pytest.approx(O.recall(mask, tm[s, :, :nt].astype(np.float32), kk),
+                                                       abs=1e-6)
 
 
 def test_dense_path_full_size_sampled():

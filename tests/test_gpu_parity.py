@@ -571,3 +571,81 @@ def test_tilemap_split_key_range(idx, heads, n_rows):
         M, _ = O.full_tilemap(f64(qp)[0, h], f64(kp)[0, h], lays[h]["lens"], w.tile, scale, rows[s, pick])
         _row_rel(gm[s, pick, :nt], M)
         assert not gm[s, :, nt:].any()
+
+
+# ------------------------------------------------ recall of the mask (a9)
+
+def _recall_rows_oracle(pred_idx, M_rows, k):
+    """Hits per row through the oracle's recall on single rows."""
+    nt = M_rows.shape[1]
+    out = []
+    for p, m in zip(pred_idx, M_rows):
+        mask = np.zeros((1, nt), bool)
+        mask[0, p[:k]] = True
+        out.append(round(O.recall(mask, m[None], k) * k))
+    return np.array(out)
+
+
+@pytest.mark.parametrize("name", ["cfg0", "ragged-d128-t128", "odd-d128-t64", "d64-t64-padded", "single-tile"])
+@pytest.mark.parametrize("kmode", ["keep", "one", "all"])
+def test_tilemap_recall(name, kmode):
+    """Recall of a predicted top-k mask against the tile map's own top-k
+    (Veda summary 2.1, Target Construction). Exact against the oracle's
+    recall applied to the GPU's map rows and mask (hits are integers; the map
+    is ranked with the same fp32 order and tie rule), and equal to the
+    oracle's recall on the fp64 oracle map wherever that row's top-k is not
+    decided by values closer than the map tolerance (1e-3 relative)."""
+    w = WL[name]
+    L = _layer(w)
+    lays, perms, n_cap, nt_cap = oracle_geometry(w)
+    q, k, _ = _inputs(w)
+    qp, _ = _permuted(L, w, q)
+    kp, _ = _permuted(L, w, k)
+    heads = list(range(w.heads))[::-1]
+    n_rows = min(l["nt"] for l in lays)
+    rows = np.stack([np.random.default_rng(30 + h).permutation(lays[h]["nt"])[:n_rows] for h in heads]).astype(np.int32)
+    kk = {"keep": oracle_k(w, lays), "one": [1] * w.heads, "all": [l["nt"] for l in lays]}[kmode]
+    k_cap = max(kk)
+    scale = 1 / math.sqrt(w.d)
+    tm = torch.empty((len(heads), n_rows, nt_cap), dtype=torch.float32, device=DEV)
+    rows_d = torch.from_numpy(rows).to(DEV)
+    V.veda_full_attn_tilemax(L, qp, kp, heads, rows_d, n_rows, scale, tm)
+    # the predicted lists: top-k of random scores with planted ties
+    rng = np.random.default_rng(9)
+    sc = rng.integers(0, 4, size=(1, w.heads, nt_cap, nt_cap)).astype(np.float32)
+    idx = torch.empty((1, w.heads, nt_cap, k_cap), dtype=torch.int32, device=DEV)
+    V.veda_topk_mask(L, torch.from_numpy(sc).to(DEV), kk, k_cap, idx)
+    hits = torch.full((len(heads), n_rows), -7, dtype=torch.int32, device=DEV)
+    rec = torch.empty(len(heads) + 1, dtype=torch.float32, device=DEV)
+    map_idx = torch.empty((len(heads), n_rows, k_cap), dtype=torch.int32, device=DEV)
+    V.veda_tilemap_recall(L, heads, rows_d, n_rows, tm, idx, kk, k_cap, hits, rec, map_idx=map_idx)
+    V.veda_check_status(L)
+    gm = tm.cpu().numpy()
+    gh, gr, gi = hits.cpu().numpy(), rec.cpu().numpy().astype(np.float64), map_idx.cpu().numpy()
+    pred_all = idx.cpu().numpy()
+    xq, xk = f64(qp), f64(kp)
+    per_head = []
+    for s, h in enumerate(heads):
+        nt, kh = lays[h]["nt"], kk[h]
+        pred = pred_all[0, h, rows[s]]
+        # exact: the oracle's ranking of the GPU's fp32 map rows
+        ref_idx, _ = O.topk_rows(gm[s, :, :nt], kh, k_cap)
+        assert np.array_equal(gi[s], ref_idx)
+        want = _recall_rows_oracle(pred, gm[s, :, :nt], kh)
+        assert np.array_equal(gh[s], want)
+        mask = np.zeros((n_rows, nt), bool)
+        for r in range(n_rows):
+            mask[r, pred[r, :kh]] = True
+        r_or = O.recall(mask, gm[s, :, :nt], kh)
+        assert gr[s] == pytest.approx(r_or, abs=1e-6)
+        per_head.append(r_or)
+        # against the fp64 oracle map, on rows whose top-k is not a near tie
+        M, _ = O.full_tilemap(xq[0, h], xk[0, h], lays[h]["lens"], w.tile, scale, rows[s])
+        want64 = _recall_rows_oracle(pred, M, kh)
+        srt = -np.sort(-M, axis=1)
+        clear = np.ones(n_rows, bool) if kh >= nt else (srt[:, kh - 1] - srt[:, kh]) > 1e-3 * srt[:, 0]
+        assert clear.any()
+        assert np.array_equal(gh[s][clear], want64[clear])
+    assert gr[-1] == pytest.approx(np.mean(per_head), abs=1e-6)
+    if kmode == "all":
+        assert (gh == np.array([[kk[h]] for h in heads])).all() and np.allclose(gr, 1.0)

@@ -6,8 +6,10 @@ pre-planned device memory pool, and real-time loops that must not enter an
 allocator between frames. For them the library keeps the embedding scratch in
 a built-in device array. This checks, through the C ABI, that two calls in a
 row (the second with different inputs, so stale scratch contents would show)
-give the regular call's scores, and that a layer too large for the built-in
-array is refused. It lives in its own file so that it runs last."""
+give the regular call's scores bit for bit (both run the same kernels on the
+same inputs), that a call after the first one changes no device memory
+reservation, and that a layer too large for the built-in array is refused.
+It lives in its own file so that it runs last."""
 import numpy as np
 import pytest
 import torch
@@ -16,12 +18,6 @@ import block_sparse_attention_24_b200 as V
 import synth
 
 pytestmark = pytest.mark.gpu
-
-
-def _row_rel_close(got, want, tol=1e-3):
-    g, w = got.double(), want.double()
-    scale = w.abs().amax(dim=-1, keepdim=True).clamp_min(1e-30)
-    return bool(((g - w).abs() <= tol * scale).all())
 
 
 def _inputs(w, nt_cap, seed):
@@ -48,7 +44,16 @@ def test_noalloc_matches_regular_call_twice():
         V.veda_tile_scores_noalloc(L, *args, synth.MLP_HIDDEN, synth.MLP_OUT, synth.SCORE_SCALE, got)
         V.veda_check_status(L)
         assert torch.isfinite(got).all()
-        assert _row_rel_close(got, want)
+        assert torch.equal(got, want)
+    # the first call on this device has set up its scratch address; later
+    # calls reserve no device memory
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    V.veda_tile_scores_noalloc(L, *args, synth.MLP_HIDDEN, synth.MLP_OUT, synth.SCORE_SCALE, got)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.equal(got, want)
 
 
 def test_noalloc_refuses_layers_beyond_its_scratch():
