@@ -1,28 +1,38 @@
 // Tile-skipping sparse attention on sm_100a (Veda summary 2.3, Hardware-
-// Efficient Implementation), one 128-row query block per CTA: each CTA walks
-// only the key/value tiles its query tiles kept; skipped tiles are never
-// loaded. Used for 64-token tiles; 128-token tiles go to the two-tile kernel
-// in attn_pair.cu.
+// Efficient Implementation) for 64-token tiles: one CTA per pair of query
+// tiles (a 128-row query block), walking the union of the two tiles' kept
+// key-tile lists two tiles at a time; tiles neither kept are never loaded.
+// 128-token tiles go to the two-tile kernel in attn_pair.cu.
+//
+// A 128 x 128 S block covers query tiles a0 (rows 0-63) and a1 (rows 64-127)
+// against two union tiles u0 (keys 0-63) and u1 (keys 64-127). Each of the
+// four 64 x 64 quarters is used when its query tile kept its key tile, and
+// its P is zero otherwise. Neighbouring query tiles keep mostly the same key
+// tiles, so the union is much shorter than the two lists together and most
+// quarters are used: with one key tile per query tile per block (the other
+// layout) only the two diagonal quarters would be.
 //
 // Roles (224 threads):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r. Reads a row
-//              of S from TMEM, keeps the row reference and sum in fp32, writes P
-//              (bf16 pairs) back into the first half of the same TMEM
-//              columns, rescales O in TMEM on the rare block whose P sum
-//              nears the fp32 range, and finally normalises O and stores it.
-//   warp 4     K producer: TMA loads of Q once and of the selected K tiles
-//              into a 3-stage ring (128B-swizzled).
+//   warps 0-3  softmax: thread r owns query row r = TMEM lane r. Reads its
+//              query tile's kept halves of a row of S from TMEM, keeps the row
+//              reference and sum in fp32, writes P (bf16 pairs, zero in the
+//              halves its query tile did not keep) back into the first half of
+//              the same TMEM columns, rescales O in TMEM on the rare block
+//              whose P sum nears the fp32 range, and finally normalises O and
+//              stores it.
+//   warp 4     K producer: TMA loads of Q once and of each step's two union
+//              K tiles into a 3-stage ring (128B-swizzled).
 //   warp 5     MMA issuer (one thread): S = Q K^T (A, B from shared memory)
 //              into one of two TMEM buffers; O += P V with P read from TMEM
 //              and V from shared memory; tcgen05.commit to mbarriers.
-//   warp 6     V producer: TMA loads of the selected V tiles, 3-stage ring.
-// K and V have their own producers so a K load never waits behind a V slot.
-// Per key block j the MMA warp queues PV_j and then S_{j+2} as soon as P_j
-// is in TMEM, so the tensor core works on them while softmax j+1 runs.
+//   warp 6     V producer: TMA loads of each step's two union V tiles.
+// Per step j the MMA warp queues PV_j and then S_{j+2} as soon as P_j is in
+// TMEM, so the tensor core works on them while softmax j+1 runs.
 //
-// Tiles of 64 tokens: a CTA still computes 128x128 blocks; its two 64-row
-// query tiles each pair with their own 64-key tile, so only the two diagonal
-// 64x64 blocks of S are used (the others are zero in P).
+// The union is walked over kept-tile bitmaps in shared memory when both lists
+// are ascending, distinct and in range (and the bitmaps fit beside the
+// rings), else by merging the lists as given; an odd union's last step loads
+// its one tile into both halves, the second kept by neither query tile.
 //
 // Every mbarrier wait is bounded (VEDA_WAIT_LIMIT_NS); on expiry the CTA
 // records VEDA_ERR_TIMEOUT, drains the copies and MMAs it issued, frees its
@@ -30,6 +40,7 @@
 #include <type_traits>
 
 #include "veda_internal.cuh"
+#include "walk.cuh"
 
 namespace veda {
 namespace {
@@ -51,13 +62,15 @@ struct AttnLayout {
   static constexpr int OFF_BAR = OFF_V + VST * KB;
   // q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], p_full[2], pv_done[2], drain
   static constexpr int NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int SMEM_ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, list check
+  static constexpr int OFF_BM = (OFF_MISC + 16 + 15) / 16 * 16;  // kept-tile bitmaps of a0 and a1
+  // dynamic shared memory with bitmaps of `words` 32-bit words each
+  static constexpr int alloc(int words) { return OFF_BM + 8 * words + 1024; }  // + 1024-byte alignment slack
 };
 
 struct AttnParams {
   int32_t k_cap;
+  int32_t bm_words;  // 32-bit words per kept-tile bitmap; 0: merge the lists
   float scale_log2;  // scale * log2(e)
   const int32_t* idx;
   __nv_bfloat16* op;    // [B, heads, n_cap, D] (permuted order), or NULL when otok is set
@@ -65,16 +78,67 @@ struct AttnParams {
   float* lse;
 };
 
-// Key tile at block j of an index row (dense path: j itself), clamped into
-// range; an out-of-range entry is reported.
-__device__ __forceinline__ int key_tile(const int32_t* row, int j, int nt, int32_t* status) {
-  if (!row) return j;
-  int t = __ldg(row + j);
-  if (t < 0 || t >= nt) {
-    report(status, VEDA_ERR_BAD_INDEX);
-    t = 0;
+// Two consecutive union tiles per step. keep bit (2*s + h): query tile s of
+// the block kept the step's tile h. An odd union's last step repeats its one
+// tile in half 1, kept by neither (its loaded values meet only zeros in P).
+template <class W>
+struct StepWalk {
+  W w;
+  __device__ bool next(int& t0, int& t1, uint32_t& keep) {
+    int t;
+    bool ma, mb;
+    if (!w.next(t, ma, mb)) return false;
+    t0 = t;
+    keep = (ma ? 1u : 0u) | (mb ? 4u : 0u);
+    if (w.next(t, ma, mb)) {
+      t1 = t;
+      keep |= (ma ? 2u : 0u) | (mb ? 8u : 0u);
+    } else {
+      t1 = t0;
+    }
+    return true;
   }
-  return t;
+};
+template <class W>
+__device__ __forceinline__ StepWalk<W> steps_of(const W& w) {
+  return StepWalk<W>{w};
+}
+
+// Maximum of one 64-key half of a row of S over its first `klen` keys.
+template <bool FULL>
+__device__ __forceinline__ float half_row_max(const uint32_t (&u)[64], int klen) {
+  float pm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 64; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float v0 = (FULL || c + i < klen) ? __uint_as_float(u[c + i]) : -INFINITY;
+      const float v1 = (FULL || c + 8 + i < klen) ? __uint_as_float(u[c + 8 + i]) : -INFINITY;
+      pm[i] = fmax3(pm[i], v0, v1);
+    }
+  return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+}
+
+// P = 2^(s*C - m) for one 64-key half as 32 bf16 pairs into pk[32h..32h+32)
+// (MUFU ex2), keys at or past `klen` zero; adds the fp32 values to acc.
+template <bool FULL>
+__device__ __forceinline__ void half_row_p(const uint32_t (&u)[64], int h, int klen, uint64_t C2, uint64_t NM,
+                                           uint64_t (&acc)[4], uint32_t (&pk)[64]) {
+#pragma unroll
+  for (int w = 0; w < 32; ++w) {
+    const uint64_t x = f2_fma(f2(__uint_as_float(u[2 * w]), __uint_as_float(u[2 * w + 1])), C2, NM);
+    float x0, x1;
+    f2_split(x, x0, x1);
+    float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+    if (!FULL) {
+      p0 = 2 * w < klen ? p0 : 0.f;
+      p1 = 2 * w + 1 < klen ? p1 : 0.f;
+    }
+    acc[w & 3] = f2_add(acc[w & 3], f2(p0, p1));
+    pk[32 * h + w] = pack_bf16x2_rn(p0, p1);
+  }
 }
 
 // Tensor maps of the permuted layout [B*heads, n_cap, d] (Q boxes of 128
@@ -89,6 +153,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ LayerGeom g,
                        const __grid_constant__ std::conditional_t<TOK, TokenMaps, PermMaps> maps,
                        const AttnParams prm) {
+  static_assert(TILE == 64, "the union walk pairs two 64-token tiles per 128-key block");
   using Lay = AttnLayout<D>;
   constexpr int NSUB = BM / TILE;
   extern __shared__ uint8_t smem_raw[];
@@ -128,15 +193,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* mma_drain = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
+  volatile int* list_bad = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 8);
+  uint32_t* bm0 = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BM);
+  uint32_t* bm1 = bm0 + prm.bm_words;
 
-  const int n = hg.k;  // key blocks (kept tiles per query tile)
-  const int32_t* lists[NSUB];
-#pragma unroll
-  for (int s = 0; s < NSUB; ++s) {
-    int a = qb * NSUB + s;
-    if (a >= nt) a = qb * NSUB;  // missing second query tile: reuse the first list
-    lists[s] = prm.idx ? prm.idx + ((long long)bh * g.nt_cap + a) * prm.k_cap : nullptr;
-  }
+  // the block's query tiles a0 = 2 qb and a1 = 2 qb + 1 (a1 may be past the
+  // head's last tile: then it keeps nothing)
+  const int a0 = qb * NSUB, a1 = a0 + 1;
+  const bool has1 = a1 < nt;
+  const int n = hg.k;
+  const int k0 = n, k1 = has1 ? n : 0;
+  const int32_t* list0 = prm.idx ? prm.idx + ((long long)bh * g.nt_cap + a0) * prm.k_cap : nullptr;
+  const int32_t* list1 = prm.idx ? prm.idx + ((long long)bh * g.nt_cap + (has1 ? a1 : a0)) * prm.k_cap : nullptr;
+  const bool try_bm = prm.idx != nullptr && prm.bm_words > 0;  // uniform over the CTA
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < Lay::NUM_BARS; ++i) {
@@ -144,15 +213,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar, (bar == p_full || bar == p_full + 1) ? 128 : 1);
     }
     *abort_flag = 0;
+    *list_bad = 0;
     fence_mbar_init();
   }
   if (warp == 5) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
+  if (try_bm) {
+    for (int i = threadIdx.x; i < 2 * prm.bm_words; i += NUM_THREADS) bm0[i] = 0u;
+    __syncthreads();
+    build_kept_bitmaps(list0, k0, list1, k1, nt, bm0, bm1, list_bad, threadIdx.x, NUM_THREADS);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const bool use_bm = try_bm && *list_bad == 0;
+  // runs fn on the step walk of this CTA's union (one walk type instantiated
+  // per call site, so only one walk's state is live)
+  auto with_steps = [&](int32_t* status, auto&& fn) {
+    if (use_bm) {
+      auto sw = steps_of(BitWalk(bm0, bm1, prm.bm_words));
+      fn(sw);
+    } else {
+      auto sw = steps_of(UnionWalk(list0, k0, list1, k1, nt, status));
+      fn(sw);
+    }
+  };
 
   if (warp == 4 || warp == 6) {
     // ----------------------------------------------------------- producers
@@ -188,25 +275,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       int issued = 0;
-      for (int t = 0; t < n; ++t) {
-        const int st = t % ST;
-        int kts[NSUB];
+      with_steps(is_k ? g.dev_status : nullptr, [&](auto& sw) {
+        int kt[2];
+        uint32_t keep;
+        for (int t = 0; sw.next(kt[0], kt[1], keep); ++t) {
+          const int st = t % ST;
+          if (t >= ST && !mbar_wait(empty + st, ((t - ST) / ST) & 1, abort_flag, g.dev_status)) break;
+          mbar_expect_tx(full + st, Lay::KB);
+          uint8_t* dst = ring + st * Lay::KB;
 #pragma unroll
-        for (int u = 0; u < NSUB; ++u) kts[u] = key_tile(lists[u], t, nt, is_k ? g.dev_status : nullptr);
-        if (t >= ST && !mbar_wait(empty + st, ((t - ST) / ST) & 1, abort_flag, g.dev_status)) break;
-        mbar_expect_tx(full + st, Lay::KB);
-        uint8_t* dst = ring + st * Lay::KB;
+          for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int u = 0; u < NSUB; ++u)
-#pragma unroll
-          for (int bx = 0; bx < D / 64; ++bx)
-            if constexpr (TOK)
-              tma_load_tile_tokens(dst + bx * BN * 128 + u * TILE * 128, map, full + st, g, hg, bx * 64, h, b,
-                                   kts[u]);
-            else
-              tma_load_3d(dst + bx * BN * 128 + u * TILE * 128, map, full + st, bx * 64, kts[u] * TILE, bh);
-        issued = t + 1;
-      }
+            for (int bx = 0; bx < D / 64; ++bx)
+              if constexpr (TOK)
+                tma_load_tile_tokens(dst + bx * BN * 128 + u * TILE * 128, map, full + st, g, hg, bx * 64, h, b,
+                                     kt[u]);
+              else
+                tma_load_3d(dst + bx * BN * 128 + u * TILE * 128, map, full + st, bx * 64, kt[u] * TILE, bh);
+          issued = t + 1;
+        }
+      });
       if (*abort_flag) {  // let every copy this warp started land before exiting
         if (is_k) mbar_wait_drain(q_full, 0, VEDA_WAIT_LIMIT_NS);
         for (int t = issued - ST < 0 ? 0 : issued - ST; t < issued; ++t)
@@ -221,6 +309,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t aQ = smem_u32(sQ);
       const uint32_t aK = smem_u32(smem + Lay::OFF_K);
       const uint32_t aV = smem_u32(smem + Lay::OFF_V);
+      // the number of steps of the walk
+      int n_steps = 0;
+      with_steps(nullptr, [&](auto& sw) {
+        int t0, t1;
+        uint32_t keep;
+        while (sw.next(t0, t1, keep)) ++n_steps;
+      });
       auto issue_s = [&](int t) -> bool {
         const int s = t & 1, st = t % KST;
         if (!mbar_wait(k_full + st, (t / KST) & 1, abort_flag, g.dev_status)) return false;
@@ -238,8 +333,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = mbar_wait(q_full, 0, abort_flag, g.dev_status);
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < 2 && t < n && ok; ++t) ok = issue_s(t);
-        for (int j = 0; j < n && ok; ++j) {
+        for (int t = 0; t < 2 && t < n_steps && ok; ++t) ok = issue_s(t);
+        for (int j = 0; j < n_steps && ok; ++j) {
           const int s = j & 1, sv = j % VST;
           if (!mbar_wait(p_full + s, (j >> 1) & 1, abort_flag, g.dev_status)) break;
           if (!mbar_wait(v_full + sv, (j / VST) & 1, abort_flag, g.dev_status)) break;
@@ -252,7 +347,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                          (j > 0 || kk > 0) ? 1u : 0u);
           umma_commit(pv_done + s);
           umma_commit(v_empty + sv);
-          if (j + 2 < n) ok = issue_s(j + 2);  // overwrites S buffer s after PV_j has read P_j
+          if (j + 2 < n_steps) ok = issue_s(j + 2);  // overwrites S buffer s after PV_j has read P_j
         }
       }
       umma_commit(mma_drain);
@@ -261,125 +356,134 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------- softmax
     const int r = threadIdx.x;                 // query row in the block
-    const int sub = r / TILE;                  // query sub-tile
+    const int sub = r / TILE;                  // the block's query tile (0 or 1)
     const int a = qb * NSUB + sub;             // query tile
-    const int32_t* my_list = (NSUB == 1 || sub == 0) ? lists[0] : lists[NSUB - 1];
     const bool row_valid = a < nt && (r % TILE) < tile_len(hg, g.T, a);
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     const float C = prm.scale_log2;
     const uint64_t C2 = f2(C, C);
+    const bool padded = hg.padded != 0;
     float m = -INFINITY, l = 0.f;
+    bool have_ref = false;  // the row's reference m is set (its first kept tile seen)
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      const int kt = key_tile(my_list, j, nt, nullptr);
-      const int klen = tile_len(hg, g.T, kt);
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, ph, abort_flag, g.dev_status))) { ok = false; break; }
-      tc_fence_after();
-      const bool full = klen == TILE;
-      float sv[TILE];
-      // the row of S_j, masked past a padded key tile's valid prefix
-      auto load_s = [&]() {
-        uint32_t u[TILE];
-        if constexpr (TILE == 128) tmem_ld128(lane_addr + s * BN, u);
-        else tmem_ld64(lane_addr + s * BN + sub * TILE, u);
-#pragma unroll
-        for (int e = 0; e < TILE; ++e) sv[e] = __uint_as_float(u[e]);
-        if (!full) {
-#pragma unroll
-          for (int c = 0; c < TILE; ++c) sv[c] = c < klen ? sv[c] : -INFINITY;
+    int n_steps = 0;
+    with_steps(nullptr, [&](auto& sw) {
+      int kt[2];
+      uint32_t keep;
+      for (int j = 0; sw.next(kt[0], kt[1], keep); ++j) {
+        n_steps = j + 1;
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        // this query tile's kept halves (uniform over the warp: a warp's rows
+        // belong to one query tile)
+        const bool kh0 = (keep >> (2 * sub)) & 1u, kh1 = (keep >> (2 * sub + 1)) & 1u;
+        const int klen0 = padded ? tile_len(hg, g.T, kt[0]) : TILE;
+        const int klen1 = padded ? tile_len(hg, g.T, kt[1]) : TILE;
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, ph, abort_flag, g.dev_status))) {
+          ok = false;
+          break;
         }
-      };
-      // row max: 8 independent 3-input max chains
-      auto row_max = [&]() -> float {
-        float pm[8];
+        tc_fence_after();
+        uint32_t pk[64];
+        // exact maximum of the kept halves' valid keys
+        auto kept_max = [&]() -> float {
+          float mx = -INFINITY;
+          if (kh0) {
+            uint32_t u[64];
+            tmem_ld64(lane_addr + s * BN, u);
+            mx = klen0 >= TILE ? half_row_max<true>(u, klen0) : half_row_max<false>(u, klen0);
+          }
+          if (kh1) {
+            uint32_t u[64];
+            tmem_ld64(lane_addr + s * BN + TILE, u);
+            mx = fmaxf(mx, klen1 >= TILE ? half_row_max<true>(u, klen1) : half_row_max<false>(u, klen1));
+          }
+          return mx;
+        };
+        // P of the kept halves against reference mref (zeros elsewhere);
+        // returns the fp32 row sum
+        auto make_p = [&](float mref) -> float {
+          const uint64_t NM = f2(-mref, -mref);
+          uint64_t acc[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) pm[i] = fmaxf(sv[i], sv[i + 8]);
+          for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
+          if (kh0) {
+            uint32_t u[64];
+            tmem_ld64(lane_addr + s * BN, u);
+            if (klen0 >= TILE) half_row_p<true>(u, 0, klen0, C2, NM, acc, pk);
+            else half_row_p<false>(u, 0, klen0, C2, NM, acc, pk);
+          } else {
 #pragma unroll
-        for (int c = 16; c < TILE; c += 16)
+            for (int w = 0; w < 32; ++w) pk[w] = 0u;
+          }
+          if (kh1) {
+            uint32_t u[64];
+            tmem_ld64(lane_addr + s * BN + TILE, u);
+            if (klen1 >= TILE) half_row_p<true>(u, 1, klen1, C2, NM, acc, pk);
+            else half_row_p<false>(u, 1, klen1, C2, NM, acc, pk);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], sv[c + i], sv[c + 8 + i]);
-        return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-      };
-      // P = 2^(s*C - mref) as bf16 pairs into pk, packed fp32x2 FMAs and
-      // MUFU ex2; returns the row sum.
-      uint32_t pk[64];  // the row of P: 128 keys as bf16 pairs
-      auto make_p = [&](float mref) -> float {
-        const uint64_t NM = f2(-mref, -mref);
-        uint64_t acc[4];
+            for (int w = 0; w < 32; ++w) pk[32 + w] = 0u;
+          }
+          float lo, hi;
+          f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
+          return lo + hi;
+        };
+        float rs = 0.f;
+        if (kh0 || kh1) {
+          // Only the row's first kept tile is max-reduced. Later tiles reuse
+          // its reference: P may exceed 1 when they hold larger logits, which
+          // fp32 and bf16 carry at full relative precision, so the reference
+          // moves only when a step's P sum nears the top of the range (rare);
+          // S_j is still in TMEM then (P is stored below), so the step is
+          // recomputed exactly.
+          if (!have_ref) {
+            m = kept_max() * C;
+            have_ref = true;
+          }
+          rs = make_p(m);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
-#pragma unroll
-        for (int w = 0; w < 64; ++w) pk[w] = 0u;
-#pragma unroll
-        for (int q = 0; q < TILE / 8; ++q) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c0 = q * 8 + 2 * e;
-            const uint64_t x = f2_fma(f2(sv[c0], sv[c0 + 1]), C2, NM);
-            float x0, x1;
-            f2_split(x, x0, x1);
-            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            if (!full) {
-              p0 = c0 < klen ? p0 : 0.f;
-              p1 = c0 + 1 < klen ? p1 : 0.f;
+          for (int w = 0; w < 64; ++w) pk[w] = 0u;
+        }
+        const bool redo = !(rs <= OVERFLOW_SUM);
+        if (__any_sync(0xffffffffu, redo)) {
+          const float mx2 = kept_max() * C;  // TMEM loads: the whole warp takes them
+          const float m_new = redo ? fmaxf(m, mx2) : m;
+          const float alpha = fast_exp2(m - m_new);
+          if (j > 0) {
+            // O must hold PV_{j-1} before it is rescaled
+            if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
+                                                   g.dev_status))) {
+              ok = false;
+              break;
             }
-            acc[e] = f2_add(acc[e], f2(p0, p1));
-            if (NSUB == 1 || sub == 0) pk[c0 / 2] = pack_bf16x2_rn(p0, p1);
-            else pk[(TILE + c0) / 2] = pack_bf16x2_rn(p0, p1);
-          }
-        }
-        const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
-        float lo, hi;
-        f2_split(f2_add(a01, a23), lo, hi);
-        return lo + hi;
-      };
-      load_s();
-      // Only the first block of a row is max-reduced. Later blocks reuse its
-      // reference: P may exceed 1 when they hold larger logits, which fp32 and
-      // bf16 carry at full relative precision, so the reference moves only
-      // when a block's P sum nears the top of the range (rare); S_j is still
-      // in TMEM then (P is stored below), so the block is recomputed exactly.
-      if (j == 0) m = row_max() * C;
-      float rs = make_p(m);
-      const bool redo = !(rs <= OVERFLOW_SUM);
-      if (__any_sync(0xffffffffu, redo)) {
-        load_s();
-        const float mx2 = row_max() * C;
-        const float m_new = redo ? fmaxf(m, mx2) : m;
-        const float alpha = fast_exp2(m - m_new);
-        if (j > 0) {
-          // O must hold PV_{j-1} before it is rescaled
-          if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
-                                                 g.dev_status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+            tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t u[32];
-            tmem_ld32(lane_addr + 2 * BN + c * 32, u);
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t u[32];
+              tmem_ld32(lane_addr + 2 * BN + c * 32, u);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(lane_addr + 2 * BN + c * 32, u);
+              for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+              tmem_st32(lane_addr + 2 * BN + c * 32, u);
+            }
           }
+          l *= alpha;
+          m = m_new;
+          if (kh0 || kh1) rs = make_p(m);
         }
-        l *= alpha;
-        m = m_new;
-        rs = make_p(m);
+        l += rs;
+        tmem_st64(lane_addr + s * BN, pk);  // P_j over the first half of S_j
+        tc_fence_before();
+        mbar_arrive(p_full + s);
       }
-      l += rs;
-      tmem_st64(lane_addr + s * BN, pk);  // P_j over the first half of S_j
-      tc_fence_before();
-      mbar_arrive(p_full + s);
-    }
+    });
     // epilogue: O / l -> bf16
-    if (ok && n > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, g.dev_status))) {
+    if (ok && n_steps > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(pv_done + ((n_steps - 1) & 1), ((n_steps - 1) >> 1) & 1, abort_flag,
+                                          g.dev_status))) {
       tc_fence_after();
-      const float inv = row_valid ? 1.0f / l : 0.f;
+      const float inv = row_valid && l > 0.f ? 1.0f / l : 0.f;
       const bool in_range = qb * BM + r < g.n_cap;
       // the row's destination: its permuted slot, or its token (padding rows
       // have none)
@@ -404,7 +508,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
       }
-      if (prm.lse && in_range) prm.lse[row0 + r] = row_valid ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
+      if (prm.lse && in_range)
+        prm.lse[row0 + r] = row_valid && l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
     }
     tc_fence_before();
   }
@@ -416,7 +521,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <int D, int TILE, bool TOK>
-cudaError_t launch_t(const LayerGeom& g0, const void* qp, const void* kp, const void* vp, const AttnParams& prm,
+cudaError_t launch_t(const LayerGeom& g0, const void* qp, const void* kp, const void* vp, const AttnParams& prm0,
                      cudaStream_t s) {
   LayerGeom g = g0;
   std::conditional_t<TOK, TokenMaps, PermMaps> maps;
@@ -431,7 +536,13 @@ cudaError_t launch_t(const LayerGeom& g0, const void* qp, const void* kp, const 
       return cudaErrorInvalidValue;
   }
   auto kern = sparse_attn_kernel<D, TILE, TOK>;
-  const int smem = AttnLayout<D>::SMEM_ALLOC;
+  AttnParams prm = prm0;
+  prm.bm_words = (g.nt_cap + 31) / 32;
+  int smem = AttnLayout<D>::alloc(prm.bm_words);
+  if (smem > 232448) {  // bitmaps do not fit beside the rings: merge the lists
+    prm.bm_words = 0;
+    smem = AttnLayout<D>::alloc(0);
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int qblocks = (g.nt_cap * TILE + BM - 1) / BM;
@@ -451,6 +562,7 @@ cudaError_t launch_sparse_attn(const LayerGeom& g, const void* qp, const void* k
                                void* o_tokens, bool tokens_in) {
   AttnParams prm;
   prm.k_cap = k_cap;
+  prm.bm_words = 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.idx = idx;
   prm.op = o_tokens ? nullptr : reinterpret_cast<__nv_bfloat16*>(op);
