@@ -42,7 +42,8 @@ import synth  # noqa: E402
 METRIC = "block-sparse attn ms/layer & effective TFLOP/s at 90% sparsity vs dense path"
 UNIT = "TFLOP/s"
 MAP_ROWS = 120          # query tiles per tile-map head (10% of 1200: sparse supervision)
-KERNELS_PER_STEP = 13   # 2 permute+TripPool, permute V, MLP + score GEMM, top-k, attention (output in token order), map sweep + finish, KL rows, KL mean, recall rows + mean
+KERNELS_FRONT_ATTN = 7  # 2 permute+TripPool, permute V, MLP + score GEMM, top-k, attention (output in token order)
+KERNELS_MAP = 6         # map sweep + finish, KL rows, KL mean, recall rows + mean
 
 
 # ------------------------------------------------------------------ ranks
@@ -66,6 +67,15 @@ def max_over_ranks(x: float, device) -> float:
         return float(x)
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device) -> float:
+    """Sum of x over all ranks (host-side bookkeeping outside the timed region)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
     return float(t.item())
 
 
@@ -155,15 +165,35 @@ def measured_peaks():
 
 # --------------------------------------------------------------- our path
 
-def build_layer(w, device, seed_offset=0):
+def layer_inputs(w, device, seed_offset=0, head_range=None):
+    """Host-side description of the benchmark layer for workload w, or
+    (head_range = (h0, h1)) of the same layer restricted to heads [h0, h1):
+    (workload, scorer weights, (q, k, v), tile-map heads, their sampled query
+    tiles). A restricted layer keeps those heads' tilings, weights, Q/K/V
+    slices and tile-map rows, so a head computes exactly what it computes in
+    the whole layer."""
+    h0, h1 = (0, w.heads) if head_range is None else head_range
+    sub = w if head_range is None else synth.head_subset(w, h0, h1)
+    heads = list(sub.tilemap_heads)
+    rows = None
+    if heads:
+        nts = [(sub.T + pt - 1) // pt * (sub.H // ph) * (sub.W // pw) for pt, ph, pw in sub.tilings]
+        rows = np.stack([synth.sample_rows(nts[h], min(MAP_ROWS, nts[h]), w.seed + h0 + h) for h in heads])
+    weights = tuple(a[h0:h1] for a in synth.mlp_weights(w))
+    q, k, v = synth.qkv(w, device, seed_offset=seed_offset)
+    if head_range is not None:
+        q, k, v = (t[:, :, h0:h1].contiguous() for t in (q, k, v))
+    return sub, weights, (q, k, v), heads, rows
+
+
+def build_layer(w, device, seed_offset=0, head_range=None):
+    """The benchmark layer (or its restriction to head_range) on the device."""
     import block_sparse_attention_24_b200 as V
     from block_sparse_attention_24_b200.layer import MapRequest, VedaLayer, device_weights
-    L = V.Layer(w.B, w.heads, w.d, w.T, w.H, w.W, w.tile, w.tilings, device=device)
-    heads = list(w.tilemap_heads)
-    rows = np.stack([synth.sample_rows(L.nt[h], min(MAP_ROWS, L.nt[h]), w.seed + h) for h in heads])
-    maps = MapRequest(heads, torch.from_numpy(rows).to(device), rows.shape[1])
-    layer = VedaLayer(L, w.keep, device_weights(synth.mlp_weights(w), device), synth.SCORE_SCALE, device, maps=maps)
-    q, k, v = synth.qkv(w, device, seed_offset=seed_offset)
+    sub, weights, (q, k, v), heads, rows = layer_inputs(w, device, seed_offset, head_range)
+    L = V.Layer(sub.B, sub.heads, sub.d, sub.T, sub.H, sub.W, sub.tile, sub.tilings, device=device)
+    maps = MapRequest(heads, torch.from_numpy(rows).to(device), rows.shape[1]) if heads else None
+    layer = VedaLayer(L, w.keep, device_weights(weights, device), synth.SCORE_SCALE, device, maps=maps)
     return V, L, layer, (q, k, v)
 
 
@@ -189,7 +219,16 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(device)
     dist_init("nccl", world)
     w = synth.config(args.config, keep=args.keep)
-    V, L, layer, (q, k, v) = build_layer(w, device, seed_offset=rank_workload_seed(rank))
+    head_range = None
+    if args.shard_heads:
+        # one layer, its heads split over the ranks (no exchange: every step is per head)
+        from block_sparse_attention_24_b200.shard import head_ranges
+        head_range = head_ranges(w.heads, world)[rank]
+        if head_range[0] == head_range[1]:
+            raise SystemExit(f"rank {rank}: no heads left for {world} ranks and {w.heads} heads")
+        V, L, layer, (q, k, v) = build_layer(w, device, head_range=head_range)
+    else:
+        V, L, layer, (q, k, v) = build_layer(w, device, seed_offset=rank_workload_seed(rank))
     stream = torch.cuda.current_stream(device)
 
     clk = ClockSampler(local).__enter__()
@@ -232,7 +271,7 @@ def run_ours(args, world, rank, local):
 
     # per-stage breakdown of the front end (separate, untimed-for-value pass)
     stage_ms = stage_breakdown(V, L, layer, q, k, v, stream)
-    grad_ms = estimator_grad_ms(layer, stream)
+    grad_ms = estimator_grad_ms(layer, stream) if layer.maps is not None else None
     cache_ms = score_cache_ms(layer, q, k, v, stream)
 
     # dense path (same kernel, every tile kept) on the same permuted tensors
@@ -255,24 +294,27 @@ def run_ours(args, world, rank, local):
     attn_tflops = eff_flops / (attn_ms / 1e3) / 1e12
     layer_ms = front_ms + attn_ms + unperm_ms
     step_ms = elapsed / args.steps * 1e3
-    value = world * eff_flops / (elapsed / args.steps) / 1e12
+    total_flops = sum_over_ranks(eff_flops, device) if args.shard_heads else world * eff_flops
+    value = total_flops / (elapsed / args.steps) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, layer, L, budget_s=args.cpu_seconds)
     traffic = load_traffic()
     hbm_stages = frontend_bandwidth(L, layer, stage_ms, unperm_ms, hbm)
     alu_stages = frontend_compute(L, layer, stage_ms, clocks.get("sm_mhz"))
-    recall90 = layer_recall(layer)
-    map_rows = int(layer.maps.n_rows)
+    recall90 = layer_recall(layer) if layer.maps is not None else None
+    map_rows = int(layer.maps.n_rows) if layer.maps is not None else MAP_ROWS
+    map_kernels = layer.maps is not None
     sp95 = run_keep(V, L, layer, q, k, v, 0.05, dense_ms, burst, stream)
     del layer, q, k, v
     torch.cuda.empty_cache()
-    others = {} if args.no_other_layers else other_layers(device, burst, stream)
+    others = {} if (args.no_other_layers or world > 1) else other_layers(device, burst, stream)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": bench_config(w, world, round(1 - kept / allp, 4), map_rows),
+        "scaling": "strong" if args.shard_heads else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": bench_config(w, world, round(1 - kept / allp, 4), map_rows, args.shard_heads),
         "attn_ms": round(attn_ms, 3), "attn_tflops": round(attn_tflops, 1),
         "attn_frac_of_burst_peak": round(attn_tflops / burst, 4),
         "attn_ms_median": round(statistics.median(attn_each), 3), "attn_ms_min": round(min(attn_each), 3),
@@ -295,7 +337,7 @@ def run_ours(args, world, rank, local):
         "hbm_stages": hbm_stages,
         "alu_stages": alu_stages,
         "e2e": e2e,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_FRONT_ATTN + (KERNELS_MAP if map_kernels else 0)) * args.steps,
         "clocks": clocks,
     }
     if cpu is not None:
@@ -346,20 +388,23 @@ def run_keep(V, L, layer, q, k, v, keep, dense_ms, burst, stream, reps=10) -> di
     k_cap = max(kk)
     idx = torch.empty((L.B, L.heads, L.nt_cap, k_cap), dtype=torch.int32, device=layer.device)
     V.veda_topk_mask(L, layer.scores, kk, k_cap, idx, None)
-    hits = torch.empty_like(layer.recall_hits)
-    rec = torch.empty_like(layer.recall)
-    layer.map_recall(idx, kk, k_cap, hits, rec)
+    rec = None
+    if layer.maps is not None:
+        hits = torch.empty_like(layer.recall_hits)
+        rec = torch.empty_like(layer.recall)
+        layer.map_recall(idx, kk, k_cap, hits, rec)
     out = torch.empty_like(layer.o)
     fn = lambda: V.veda_sparse_attn_unpermute(L, layer.qp, layer.kp, layer.vp, idx, kk, k_cap, layer.attn_scale, out)
     mean_ms, min_ms = time_launches(fn, stream, reps)
     V.veda_check_status(L)
     kept, allp = kept_pairs(L, layer, idx, kk)
     tf = 4.0 * L.d * kept / (mean_ms / 1e3) / 1e12
-    r = rec.cpu().tolist()
+    r = rec.cpu().tolist() if rec is not None else None
     return {"keep": keep, "k": kk[0] if len(set(kk)) == 1 else kk, "sparsity": round(1 - kept / allp, 4),
             "attn_ms": round(mean_ms, 3), "attn_ms_min": round(min_ms, 3), "attn_tflops": round(tf, 1),
             "attn_frac_of_burst_peak": round(tf / burst, 4), "speedup_vs_dense": round(dense_ms / mean_ms, 2),
-            "recall": {"mean": round(r[-1], 4), "per_head": {str(h): round(x, 4) for h, x in zip(layer.maps.heads, r[:-1])}}}
+            "recall": None if r is None else
+            {"mean": round(r[-1], 4), "per_head": {str(h): round(x, 4) for h, x in zip(layer.maps.heads, r[:-1])}}}
 
 
 def other_layers(device, burst, stream) -> dict:
@@ -516,14 +561,16 @@ def run_e2e(V, L, layer, q, k, v, device, eff_flops, args):
             "copies": "overlapped with the kernels of the neighbouring steps (two copy streams)"}
 
 
-def bench_config(w, world, sparsity, map_rows) -> dict:
+def bench_config(w, world, sparsity, map_rows, shard_heads=False) -> dict:
     """The workload description both arms print."""
     qkv_mb = w.B * w.N * w.heads * w.d * 2 / 1e6
     return {"workload": w.name, "model": "none (one attention layer, synthetic activations)",
             "global_batch": w.B * world, "seq_len": w.N, "heads": w.heads, "head_dim": w.d,
             "tile": w.tile, "keep": w.keep, "sparsity": sparsity,
             "tilemap": {"heads": list(w.tilemap_heads), "query_tiles_per_head": int(map_rows)},
-            "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
+            "parallelism": ("single GPU" if world == 1 else
+                            f"one layer, heads split over {world} GPUs (no exchange)" if shard_heads else
+                            "independent layer per GPU"),
             "l2": (f"inputs larger than L2 (each of Q/K/V is {qkv_mb:.0f} MB)" if qkv_mb > 126 else
                    f"inputs fit in L2 (each of Q/K/V is {qkv_mb:.0f} MB); parity-size layer, not the benchmark layer")}
 
@@ -756,6 +803,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-layers", action="store_true", help="skip the 24,576- and 80,640-token attention timings")
     ap.add_argument("--sweep", action="store_true", help="head-group token/sparsity sweep instead of the step")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="N>1: one layer with its heads split over the ranks (strong scaling) instead of an "
+                         "independent layer per rank")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps are required")

@@ -119,6 +119,17 @@ def custom(name: str, B: int, heads: int, d: int, T: int, H: int, W: int, tile: 
                     tilemap_heads=tuple(tilemap_heads), k_fixed=k_fixed)
 
 
+def head_subset(w: Workload, h0: int, h1: int) -> Workload:
+    """The same layer restricted to heads [h0, h1): their tilings, and the
+    tile-map heads among them renumbered from 0. The tensors and weights of
+    the subset are the full layer's (slice qkv() and mlp_weights() by head);
+    the seed stays the full layer's."""
+    if not (0 <= h0 < h1 <= w.heads):
+        raise ValueError(f"head range [{h0}, {h1}) outside [0, {w.heads})")
+    return replace(w, name=f"{w.name}-heads{h0}-{h1}", heads=h1 - h0, tilings=w.tilings[h0:h1],
+                   tilemap_heads=tuple(h - h0 for h in w.tilemap_heads if h0 <= h < h1))
+
+
 # ---------------------------------------------------------------------------
 # random tensors
 # ---------------------------------------------------------------------------
