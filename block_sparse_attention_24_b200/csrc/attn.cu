@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       uint8_t* ring = smem + (is_k ? Lay::OFF_K : Lay::OFF_V);
-      constexpr int ST = KST;  // == VST
+      const int ST = is_k ? KST : VST;  // this producer's ring depth
       tma_prefetch_desc(map);
       if (is_k) {
         tma_prefetch_desc(qmap);

@@ -3,9 +3,12 @@ loss (veda_estimator_grad) against the fp64 oracle (estimator_grad, pinned by
 finite differences in test_oracle.py), on small layers, on sampled query
 tiles, with the tile map from the library's own kernel and with random maps.
 
-Tolerance: each gradient array within 2e-3 of the largest oracle gradient
-of its side (fp32 sums of up to nt * rows terms against fp64); the loss
-within 1e-4 relative."""
+Tolerance: each gradient array within 1e-4 of the largest oracle gradient
+of its side. The GPU sums up to nt * rows fp32 terms per weight in a fixed
+order (unit roundoff u = 6e-8); for terms of mixed sign the error grows like
+sqrt(n) * u, about 2e-5 of the largest term at n = 1.4e5 (the 153,600-token
+layer's 120 rows x 1,200 tiles), and the largest observed on these layers
+was 1e-5. The loss within 1e-4 relative."""
 import math
 
 import numpy as np
@@ -85,7 +88,7 @@ def _case(w, heads, n_rows, map_kind, tied=False, seed=0):
         scale_side = max(np.abs(ref[4 * side + i]).max() for i in range(4))
         for i in range(4 * side, 4 * side + 4):
             err = np.abs(got[i] - ref[i]).max()
-            assert err <= 2e-3 * scale_side, (NAMES[i], err, scale_side)
+            assert err <= 1e-4 * scale_side, (NAMES[i], err, scale_side)
     assert float(loss.item()) == pytest.approx(float(np.mean(losses)), rel=1e-4)
     return L, (dq, dk, Wt, heads, T(rows), n_rows, tm, ws), grads
 
