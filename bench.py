@@ -591,13 +591,14 @@ def layout_sparsity(w) -> float:
 
 
 def kernel_source_hash() -> str:
-    """Hash of the attention kernel's device source: attn_pair.cu and the
-    device-code part of veda_internal.cuh (its host launcher declarations at
-    the end change with unrelated entry points)."""
+    """Hash of the attention kernel's device source: attn_pair.cu, walk.cuh
+    and the device-code part of veda_internal.cuh (its host launcher
+    declarations at the end change with unrelated entry points)."""
     import hashlib
     csrc = os.path.join(ROOT, "block_sparse_attention_24_b200", "csrc")
     hsh = hashlib.sha256()
     hsh.update(open(os.path.join(csrc, "attn_pair.cu"), "rb").read())
+    hsh.update(open(os.path.join(csrc, "walk.cuh"), "rb").read())
     hdr = open(os.path.join(csrc, "veda_internal.cuh"), "rb").read()
     hsh.update(hdr.split(b"// Host-side launchers")[0])
     return hsh.hexdigest()[:16]

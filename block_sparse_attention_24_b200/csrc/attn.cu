@@ -23,11 +23,12 @@
 //   warp 4     K producer: TMA loads of Q once and of each step's two union
 //              K tiles into a 3-stage ring (128B-swizzled).
 //   warp 5     MMA issuer (one thread): S = Q K^T (A, B from shared memory)
-//              into one of two TMEM buffers; O += P V with P read from TMEM
+//              into one of NS = 3 TMEM buffers; O += P V with P read from TMEM
 //              and V from shared memory; tcgen05.commit to mbarriers.
 //   warp 6     V producer: TMA loads of each step's two union V tiles.
-// Per step j the MMA warp queues PV_j and then S_{j+2} as soon as P_j is in
-// TMEM, so the tensor core works on them while softmax j+1 runs.
+// Per step j the MMA warp queues PV_j and then S_{j+3} as soon as P_j is in
+// TMEM, so the tensor core works on them while softmax j+1 runs, and the
+// next steps' S are already computed when their softmax starts.
 //
 // The union is walked over kept-tile bitmaps in shared memory when both lists
 // are ascending, distinct and in range (and the bitmaps fit beside the
@@ -49,7 +50,8 @@ constexpr int BM = 128;               // query rows per CTA
 constexpr int BN = 128;               // keys per block
 constexpr int KST = 3, VST = 3;       // K and V ring stages
 constexpr float OVERFLOW_SUM = 1.8446744e19f;  // 2^64: a block's P sum above this moves the reference
-constexpr uint32_t TMEM_COLS = 512;   // S0 [0,128), S1 [128,256), O [256, 256+D)
+constexpr int NS = 3;                 // S buffers in TMEM: the MMA runs NS steps ahead of the softmax
+constexpr uint32_t TMEM_COLS = 512;   // S_0 .. S_{NS-1} at [128 s, 128 s + 128), then O [128 NS, 128 NS + D)
 constexpr int NUM_THREADS = 224;
 
 template <int D>
@@ -60,8 +62,8 @@ struct AttnLayout {
   static constexpr int OFF_K = OFF_Q + QB;
   static constexpr int OFF_V = OFF_K + KST * KB;
   static constexpr int OFF_BAR = OFF_V + VST * KB;
-  // q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1;
+  // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[NS], p_full[NS], pv_done[NS], drain
+  static constexpr int NUM_BARS = 1 + 2 * KST + 2 * VST + 3 * NS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, list check
   static constexpr int OFF_BM = (OFF_MISC + 16 + 15) / 16 * 16;  // kept-tile bitmaps of a0 and a1
   // dynamic shared memory with bitmaps of `words` 32-bit words each
@@ -187,10 +189,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* k_empty = k_full + KST;
   uint64_t* v_full = k_empty + KST;
   uint64_t* v_empty = v_full + VST;
-  uint64_t* s_full = v_empty + VST;  // [2]
-  uint64_t* p_full = s_full + 2;     // [2], 128 arrivals
-  uint64_t* pv_done = p_full + 2;    // [2]
-  uint64_t* mma_drain = pv_done + 2;
+  uint64_t* s_full = v_empty + VST;  // [NS]
+  uint64_t* p_full = s_full + NS;    // [NS], 128 arrivals
+  uint64_t* pv_done = p_full + NS;   // [NS]
+  uint64_t* mma_drain = pv_done + NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
   volatile int* list_bad = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 8);
@@ -210,7 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < Lay::NUM_BARS; ++i) {
       uint64_t* bar = bars + i;
-      mbar_init(bar, (bar == p_full || bar == p_full + 1) ? 128 : 1);
+      mbar_init(bar, (bar >= p_full && bar < p_full + NS) ? 128 : 1);
     }
     *abort_flag = 0;
     *list_bad = 0;
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         while (sw.next(t0, t1, keep)) ++n_steps;
       });
       auto issue_s = [&](int t) -> bool {
-        const int s = t & 1, st = t % KST;
+        const int s = t % NS, st = t % KST;
         if (!mbar_wait(k_full + st, (t / KST) & 1, abort_flag, g.dev_status)) return false;
         tc_fence_after();
 #pragma unroll
@@ -333,21 +335,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = mbar_wait(q_full, 0, abort_flag, g.dev_status);
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < 2 && t < n_steps && ok; ++t) ok = issue_s(t);
+        for (int t = 0; t < NS && t < n_steps && ok; ++t) ok = issue_s(t);
         for (int j = 0; j < n_steps && ok; ++j) {
-          const int s = j & 1, sv = j % VST;
-          if (!mbar_wait(p_full + s, (j >> 1) & 1, abort_flag, g.dev_status)) break;
+          const int s = j % NS, sv = j % VST;
+          if (!mbar_wait(p_full + s, (j / NS) & 1, abort_flag, g.dev_status)) break;
           if (!mbar_wait(v_full + sv, (j / VST) & 1, abort_flag, g.dev_status)) break;
           tc_fence_after();
           // P_j sits in the first 64 columns of S buffer s (two bf16 per column)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            umma_bf16_ts(tmem + 2 * BN, tmem + s * BN + kk * 8,
+            umma_bf16_ts(tmem + NS * BN, tmem + s * BN + kk * 8,
                          sdesc_sw128(aV + sv * Lay::KB + kk * 2048, BN * 128, 1024), idesc_o,
                          (j > 0 || kk > 0) ? 1u : 0u);
           umma_commit(pv_done + s);
           umma_commit(v_empty + sv);
-          if (j + 2 < n_steps) ok = issue_s(j + 2);  // overwrites S buffer s after PV_j has read P_j
+          if (j + NS < n_steps) ok = issue_s(j + NS);  // overwrites S buffer s after PV_j has read P_j
         }
       }
       umma_commit(mma_drain);
@@ -372,8 +374,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t keep;
       for (int j = 0; sw.next(kt[0], kt[1], keep); ++j) {
         n_steps = j + 1;
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+        const int s = j % NS;
+        const uint32_t ph = (j / NS) & 1;
         // this query tile's kept halves (uniform over the warp: a warp's rows
         // belong to one query tile)
         const bool kh0 = (keep >> (2 * sub)) & 1u, kh1 = (keep >> (2 * sub + 1)) & 1u;
@@ -407,23 +409,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint64_t acc[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[e] = f2(0.f, 0.f);
-          if (kh0) {
+          if (kh0 && kh1) {  // both halves: one TMEM load of the whole row
+            uint32_t u[BN];
+            tmem_ld128(lane_addr + s * BN, u);
+            const uint32_t (&u0)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&u[0]);
+            const uint32_t (&u1)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&u[64]);
+            if (klen0 >= TILE) half_row_p<true>(u0, 0, klen0, C2, NM, acc, pk);
+            else half_row_p<false>(u0, 0, klen0, C2, NM, acc, pk);
+            if (klen1 >= TILE) half_row_p<true>(u1, 1, klen1, C2, NM, acc, pk);
+            else half_row_p<false>(u1, 1, klen1, C2, NM, acc, pk);
+          } else if (kh0) {
             uint32_t u[64];
             tmem_ld64(lane_addr + s * BN, u);
             if (klen0 >= TILE) half_row_p<true>(u, 0, klen0, C2, NM, acc, pk);
             else half_row_p<false>(u, 0, klen0, C2, NM, acc, pk);
-          } else {
 #pragma unroll
-            for (int w = 0; w < 32; ++w) pk[w] = 0u;
-          }
-          if (kh1) {
+            for (int w = 0; w < 32; ++w) pk[32 + w] = 0u;
+          } else {
             uint32_t u[64];
             tmem_ld64(lane_addr + s * BN + TILE, u);
             if (klen1 >= TILE) half_row_p<true>(u, 1, klen1, C2, NM, acc, pk);
             else half_row_p<false>(u, 1, klen1, C2, NM, acc, pk);
-          } else {
 #pragma unroll
-            for (int w = 0; w < 32; ++w) pk[32 + w] = 0u;
+            for (int w = 0; w < 32; ++w) pk[w] = 0u;
           }
           float lo, hi;
           f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float alpha = fast_exp2(m - m_new);
           if (j > 0) {
             // O must hold PV_{j-1} before it is rescaled
-            if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
+            if (!__all_sync(0xffffffffu, mbar_wait(pv_done + (j - 1) % NS, ((j - 1) / NS) & 1, abort_flag,
                                                    g.dev_status))) {
               ok = false;
               break;
@@ -462,10 +470,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t u[32];
-              tmem_ld32(lane_addr + 2 * BN + c * 32, u);
+              tmem_ld32(lane_addr + NS * BN + c * 32, u);
 #pragma unroll
               for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-              tmem_st32(lane_addr + 2 * BN + c * 32, u);
+              tmem_st32(lane_addr + NS * BN + c * 32, u);
             }
           }
           l *= alpha;
@@ -480,7 +488,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     });
     // epilogue: O / l -> bf16
     if (ok && n_steps > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(pv_done + ((n_steps - 1) & 1), ((n_steps - 1) >> 1) & 1, abort_flag,
+        __all_sync(0xffffffffu, mbar_wait(pv_done + (n_steps - 1) % NS, ((n_steps - 1) / NS) & 1, abort_flag,
                                           g.dev_status))) {
       tc_fence_after();
       const float inv = row_valid && l > 0.f ? 1.0f / l : 0.f;
@@ -497,7 +505,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
-        tmem_ld32(lane_addr + 2 * BN + c * 32, u);
+        tmem_ld32(lane_addr + NS * BN + c * 32, u);
         uint32_t o[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
