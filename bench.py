@@ -155,6 +155,11 @@ class ClockSampler:
                 "period_ms": 100}
 
 
+def measured_clock_max():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    return json.load(open(p)).get("sm_max_mhz") if os.path.exists(p) else None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -443,6 +448,10 @@ def frontend_compute(L, layer, stage_ms, sm_mhz) -> dict:
     the instruction issue rate (148 SMs x 4 schedulers x 1 warp instruction
     per clock) for its counting loop (2 integer instructions per key and
     bisection step, 32 steps, keys padded to the register layout)."""
+    clock_kind = "median SM clock sampled in the timed region"
+    if not sm_mhz:   # no sample in a short timed region: the GPU's maximum clock
+        sm_mhz = measured_clock_max()
+        clock_kind = "maximum SM clock (no sample in the timed region)"
     if not sm_mhz:
         return {}
     f = sm_mhz * 1e6
@@ -456,7 +465,7 @@ def frontend_compute(L, layer, stage_ms, sm_mhz) -> dict:
     issue = rows * 32 * 2 * kpl
     issue_peak = 148 * 4 * f
     ts, tk = stage_ms["tile_scores"] / 1e3, stage_ms["topk"] / 1e3
-    return {"clock_mhz": sm_mhz,
+    return {"clock_mhz": sm_mhz, "clock": clock_kind,
             "tile_scores": {"bound": "fp32 fma", "flop": mlp + gemm, "ms": stage_ms["tile_scores"],
                             "tflops": round((mlp + gemm) / ts / 1e12, 2), "peak_tflops": round(ffma_peak / 1e12, 1),
                             "frac": round((mlp + gemm) / ts / ffma_peak, 3)},
