@@ -109,6 +109,12 @@ def test_full_layer_sampled(name):
     V.veda_permute(L, o_sep, layer.op, inverse=True)
     torch.cuda.synchronize()
     assert torch.equal(layer.o, o_sep)
+    # and a second launch repeats the first bit for bit (a race between the
+    # kernel's roles would show here first: thousands of CTAs)
+    op_first = layer.op.clone()
+    layer.attend_permuted()
+    torch.cuda.synchronize()
+    assert torch.equal(layer.op, op_first)
 
     # tile map and KL on the benchmark's sampled heads and query tiles
     m = layer.maps

@@ -418,20 +418,39 @@ def test_sparse_attention_wide_logit_range(name, order):
     _attention_case(WL[name], dense=True, key_tile_gain=gain)
 
 
-def test_sparse_attention_deterministic():
-    w = WL["ragged-d128-t128"]
+@pytest.mark.parametrize("name", list(WL))
+@pytest.mark.parametrize("dense", [False, True])
+def test_sparse_attention_deterministic(name, dense):
+    """Repeated calls give the same bits: the kernels sum in a fixed order, so
+    any difference is a race (a buffer read before the MMA or softmax that
+    writes it has finished)."""
+    w = WL[name]
     L = _layer(w)
+    lays, _, _, nt_cap = oracle_geometry(w)
     q, k, v = _inputs(w)
     qp, _ = _permuted(L, w, q)
     kp, _ = _permuted(L, w, k)
     vp, _ = _permuted(L, w, v)
+    ks = oracle_k(w, lays)
+    k_cap = max(ks)
+    idx = np.full((w.B, w.heads, nt_cap, k_cap), -1, np.int32)
+    for b in range(w.B):
+        for h in range(w.heads):
+            nt = lays[h]["nt"]
+            idx[b, h, :nt] = synth.random_index_lists(nt, nt, ks[h], k_cap, seed=7 + 100 * b + h)
+    idx_d = torch.from_numpy(idx).to(DEV)
     outs = []
-    for _ in range(2):
-        op = torch.empty_like(qp)
-        V.veda_sparse_attn(L, qp, kp, vp, None, None, 0, 0.1, op)
+    for _ in range(4):
+        op = torch.zeros_like(qp)
+        if dense:
+            V.veda_sparse_attn(L, qp, kp, vp, None, None, 0, 0.1, op)
+        else:
+            V.veda_sparse_attn(L, qp, kp, vp, idx_d, ks, k_cap, 0.1, op)
         outs.append(op)
     torch.cuda.synchronize()
-    assert torch.equal(outs[0], outs[1])
+    V.veda_check_status(L)
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
 
 
 def test_sparse_attention_bad_index_reported():
